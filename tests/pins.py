@@ -1,0 +1,393 @@
+"""Independent checks that pin the CPU oracle to the pages and to mathematics.
+
+Each ``check_*`` function takes the oracle function under test as an argument
+and raises ``AssertionError`` when it disagrees with something other than
+itself: a pure-Python brute force written from the definition, a library
+routine on a special case, a closed form, or a worked number from the pages
+(fixtures under ``tests/golden``).  ``test_oracle_pins.py`` runs them on the
+oracle; ``test_oracle_mutations.py`` runs them on copies of the oracle with a
+planted mistake and expects them to fail.
+"""
+from __future__ import annotations
+
+import collections
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- route ----
+def brute_topk(row, k, allowed=None):
+    """Repeatedly take the largest remaining logit, lowest index first among equals."""
+    left = [e for e in range(len(row)) if allowed is None or allowed[e]]
+    out = []
+    for _ in range(k):
+        best = left[0]
+        for e in left[1:]:
+            if row[e] > row[best]:
+                best = e
+        out.append(best)
+        left.remove(best)
+    return out
+
+
+def brute_softmax(row):
+    m = max(float(v) for v in row)
+    z = [math.exp(float(v) - m) for v in row]
+    s = math.fsum(z)
+    return [v / s for v in z]
+
+
+def check_route_brute(route_topk, seed=0):
+    rng = np.random.default_rng(seed)
+    for T, E, k in [(7, 8, 3), (5, 16, 5), (4, 6, 6), (9, 33, 4)]:
+        # few distinct values -> many ties
+        logits = rng.integers(-2, 3, size=(T, E)).astype(np.float32) * np.float32(0.5)
+        idx, w = route_topk(logits, k)
+        for t in range(T):
+            exp_idx = brute_topk(list(logits[t]), k)
+            assert list(idx[t]) == exp_idx, (t, list(idx[t]), exp_idx)
+            p = brute_softmax(logits[t])
+            np.testing.assert_allclose(w[t], [p[e] for e in exp_idx], rtol=1e-13)
+
+
+def check_route_library(route_topk, seed=1):
+    import torch
+    rng = np.random.default_rng(seed)
+    logits = rng.standard_normal((64, 256)).astype(np.float32)
+    assert all(len(np.unique(r)) == r.size for r in logits)      # distinct within each row
+    idx, w = route_topk(logits, 8)
+    lt = torch.from_numpy(logits.astype(np.float64))
+    tv, ti = torch.topk(lt, 8, dim=1, largest=True, sorted=True)
+    assert np.array_equal(idx, ti.numpy().astype(np.int32))
+    p = torch.softmax(lt, dim=1).numpy()
+    np.testing.assert_allclose(w, np.take_along_axis(p, ti.numpy(), 1), rtol=1e-12)
+
+
+def check_route_special(route_topk):
+    # all equal -> lowest indices, weight 1/E
+    idx, w = route_topk(np.full((3, 10), 0.25, np.float32), 4)
+    assert np.array_equal(idx, np.tile(np.arange(4), (3, 1)))
+    np.testing.assert_allclose(w, 0.1, rtol=1e-14)
+    # k = E -> a full permutation sorted by logit
+    rng = np.random.default_rng(2)
+    lg = rng.standard_normal((5, 12)).astype(np.float32)
+    idx, w = route_topk(lg, 12)
+    for t in range(5):
+        assert sorted(idx[t].tolist()) == list(range(12))
+        assert np.all(np.diff(lg[t][idx[t]]) <= 0)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-14)
+    # huge logits: the max subtraction keeps exp finite
+    idx, w = route_topk(np.array([[1000.0, 999.0, 0.0, -1000.0]], np.float32), 2)
+    assert idx.tolist() == [[0, 1]]
+    e1 = math.exp(-1.0)
+    np.testing.assert_allclose(w[0], [1 / (1 + e1 + math.exp(-1000)), e1 / (1 + e1)], rtol=1e-14)
+    # renormalised weights sum to one and keep their ratios
+    idx, w = route_topk(lg, 3, renormalize=True)
+    _, w0 = route_topk(lg, 3)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(w * w0.sum(axis=1, keepdims=True), w0, rtol=1e-13)
+
+
+def check_route_groups(route_topk):
+    g = golden("p4_group_limited.json")
+    for c in g["cases"]:
+        lg = np.asarray([c["logits"]], np.float32)
+        idx, w = route_topk(lg, c["k"], c["n_groups"], c["groups_per_token"])
+        assert idx[0].tolist() == c["idx"], (c["note"], idx[0].tolist())
+        idx_u, _ = route_topk(lg, c["k"])
+        assert idx_u[0].tolist() == c["idx_unconstrained"]
+        p = brute_softmax(lg[0])             # softmax over all experts
+        np.testing.assert_allclose(w[0], [p[e] for e in c["idx"]], rtol=1e-13)
+    # brute force: keep best groups by max logit, then plain top-k over their experts
+    rng = np.random.default_rng(3)
+    for G, gs, gpt, k in [(4, 4, 2, 3), (8, 2, 3, 5), (2, 8, 1, 8)]:
+        E = G * gs
+        lg = rng.integers(-3, 4, size=(20, E)).astype(np.float32)
+        idx, _ = route_topk(lg, k, G, gpt)
+        for t in range(20):
+            score = [max(lg[t][g * gs:(g + 1) * gs]) for g in range(G)]
+            kept = brute_topk(score, gpt)
+            allowed = [(e // gs) in kept for e in range(E)]
+            assert idx[t].tolist() == brute_topk(list(lg[t]), k, allowed)
+        # keeping every group is plain top-k
+        assert np.array_equal(route_topk(lg, k, G, G)[0], route_topk(lg, k)[0])
+
+
+# ----------------------------------------------------------------- hist ----
+def check_hist(demand_hist, seed=4):
+    rng = np.random.default_rng(seed)
+    for T, k, E in [(1, 1, 1), (50, 3, 7), (300, 8, 64)]:
+        idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+        c = demand_hist(idx, E)
+        ref = collections.Counter(int(v) for v in idx.ravel())
+        assert [int(c[e]) for e in range(E)] == [ref.get(e, 0) for e in range(E)]
+        assert int(np.sum(c)) == T * k
+
+
+# --------------------------------------------------------------- assign ----
+def check_assign_hand(replica_assign):
+    g = golden("metro_greedy_hand.json")
+    slot, rank, act = replica_assign(np.asarray(g["counts"]), np.asarray(g["replica_offsets"]),
+                                     np.asarray(g["replica_slots"]), np.asarray(g["slot_rank"]), g["R"])
+    assert slot.tolist() == g["expert_slot"]
+    assert rank.tolist() == g["expert_rank"]
+    assert act.tolist() == g["rank_active"]
+
+
+def toy_instance():
+    g = golden("p1_toy_assignment.json")
+    R, E = g["gpus"], g["experts"]
+    counts = np.full(E, g["tokens_per_expert"])
+    offsets = np.arange(0, 2 * E + 1, 2)
+    slots = np.arange(2 * E)
+    slot_rank = np.array([[e, (e + 1) % R] for e in range(E)]).ravel()
+    return g, counts, offsets, slots, slot_rank, R
+
+
+def check_assign_toy(replica_assign, token_balanced_active):
+    g, counts, off, slots, sr, R = toy_instance()
+    assert int(counts.sum()) == g["tokens"]
+    _, _, act = replica_assign(counts, off, slots, sr, R)
+    assert int(act.max()) == g["metro_max_active_per_gpu"]
+    tb = token_balanced_active(counts, off, slots, sr, R)
+    assert tb.tolist() == [g["token_balanced_active_per_gpu"]] * R
+    # the page's "halves the expert-weight loading term"
+    assert int(tb.max()) == 2 * int(act.max())
+
+
+def check_assign_closed_forms(replica_assign, seed=5):
+    rng = np.random.default_rng(seed)
+    for E, R in [(16, 4), (64, 8), (37, 5)]:
+        counts = rng.integers(0, 3, size=E)
+        # one replica per expert: the identity map
+        sr = rng.integers(0, R, size=E)
+        slot, rank, act = replica_assign(counts, np.arange(E + 1), np.arange(E), sr, R)
+        for e in range(E):
+            assert (slot[e], rank[e]) == ((e, sr[e]) if counts[e] else (-1, -1))
+        # every expert on every rank: greedy reaches ceil(A / R), the optimum
+        off = np.arange(0, E * R + 1, R)
+        slots = np.arange(E * R)
+        sr_full = np.tile(np.arange(R), E)
+        _, _, act = replica_assign(counts, off, slots, sr_full, R)
+        A = int(np.count_nonzero(counts))
+        assert int(act.max()) == -(-A // R)
+        assert int(act.sum()) == A
+
+
+def check_assign_brute(replica_assign, optimal_max_active, seed=6):
+    """Greedy is feasible and never beats the brute-force optimum; on a fixed
+    family of tiny instances it also matches a pure-Python greedy."""
+    rng = np.random.default_rng(seed)
+    gaps = []
+    for _ in range(60):
+        E, R = int(rng.integers(1, 8)), int(rng.integers(1, 5))
+        reps = [sorted(rng.choice(R, size=int(rng.integers(1, min(R, 3) + 1)), replace=False).tolist())
+                for _ in range(E)]
+        off = np.zeros(E + 1, np.int64)
+        off[1:] = np.cumsum([len(r) for r in reps])
+        sr = np.asarray([r for rr in reps for r in rr], np.int64)
+        slots = np.arange(sr.shape[0])
+        counts = rng.integers(0, 3, size=E)
+        slot, rank, act = replica_assign(counts, off, slots, sr, R)
+        load = [0] * R
+        for e in range(E):
+            if counts[e]:
+                cands = list(range(off[e], off[e + 1]))
+                s = min(cands, key=lambda s: (load[sr[s]], sr[s], s))
+                assert slot[e] == s and rank[e] == sr[s]
+                load[sr[s]] += 1
+            else:
+                assert slot[e] == -1
+        opt = optimal_max_active(counts, off, slots, sr, R)
+        assert int(act.max() if R else 0) >= opt
+        if opt:
+            gaps.append(act.max() / opt - 1.0)
+    return float(np.mean(gaps)) if gaps else 0.0
+
+
+# --------------------------------------------------------------- layout ----
+def brute_layout(idx, w, expert_rank, tokens_per_rank, R, mode, rpg=0):
+    """Pure-Python layout straight from the row definitions."""
+    T, k = len(idx), len(idx[0])
+    rows = []                      # (dst, [e,] t, coef)
+    if mode == 0:                  # PER_PICK: (dst, e, t)
+        for d in range(R):
+            for e in sorted({int(x) for x in np.ravel(idx)}):
+                if expert_rank[e] != d:
+                    continue
+                for t in range(T):
+                    for j in range(k):
+                        if idx[t][j] == e:
+                            rows.append((d, t, float(w[t][j])))
+    else:                          # DEDUP / TWO_HOP rank rows: (dst, t)
+        for d in range(R):
+            for t in range(T):
+                ws = [float(w[t][j]) for j in range(k) if expert_rank[idx[t][j]] == d]
+                if ws:
+                    rows.append((d, t, math.fsum(ws)))
+    out = {"row_token": [r[1] for r in rows], "row_dst": [r[0] for r in rows],
+           "row_coef": [r[2] for r in rows]}
+    out["rank_offsets"] = [sum(1 for r in rows if r[0] < d) for d in range(R + 1)]
+    tr = [[i for i, r in enumerate(rows) if r[1] == t] for t in range(T)]
+    out["token_rows"] = [x + [-1] * (k - len(x)) for x in tr]
+    sc = [[0] * R for _ in range(R)]
+    for d, t, _ in rows:
+        sc[t // tokens_per_rank][d] += 1
+    out["send_counts"] = sc
+    if mode == 2:
+        G = R // rpg
+        h1 = [(g, t) for g in range(G) for t in range(T)
+              if any(expert_rank[idx[t][j]] // rpg == g for j in range(k))]
+        out["hop1_row_token"] = [t for _, t in h1]
+        out["group_offsets"] = [sum(1 for g2, _ in h1 if g2 < g) for g in range(G + 1)]
+        tg = [[i for i, (g, t2) in enumerate(h1) if t2 == t] for t in range(T)]
+        out["token_groups"] = [x + [-1] * (k - len(x)) for x in tg]
+        out["hop2_src_row"] = [h1.index((d // rpg, t)) for d, t, _ in rows]
+    return out
+
+
+def tiny_routing(seed, T, E, k, R, skew=False):
+    rng = np.random.default_rng(seed)
+    p = None
+    if skew:
+        p = 1.0 / (1.0 + np.arange(E))
+        p = p / p.sum()
+    idx = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    w = rng.uniform(0.01, 1.0, size=(T, k))
+    expert_rank = rng.integers(0, R, size=E).astype(np.int32)
+    return idx, w, expert_rank
+
+
+def check_layout_brute(build_layout):
+    cases = [(13, 8, 3, 4, 1, 0), (24, 16, 4, 8, 2, 0), (10, 6, 6, 2, 1, 0), (1, 4, 2, 4, 1, 0),
+             (32, 12, 4, 6, 3, 1)]
+    for seed, (T, E, k, R, trp, skew) in enumerate(cases):
+        Tr = -(-T // R)
+        idx, w, er = tiny_routing(seed, T, E, k, R, skew=bool(skew))
+        for mode in (0, 1, 2):
+            rpg = 2 if R % 2 == 0 else 1
+            L = build_layout(idx, w, er, Tr, R, mode, ranks_per_group=rpg)
+            B = brute_layout(idx.tolist(), w, er.tolist(), Tr, R, mode, rpg)
+            assert L["row_token"].tolist() == B["row_token"], (seed, mode)
+            assert L["row_dst"].tolist() == B["row_dst"]
+            np.testing.assert_allclose(L["row_coef"], B["row_coef"], rtol=1e-13)
+            assert L["rank_offsets"].tolist() == B["rank_offsets"]
+            assert L["token_rows"].tolist() == B["token_rows"]
+            assert L["send_counts"].tolist() == B["send_counts"]
+            assert int(L["num_rows"]) == len(B["row_token"])
+            if mode == 2:
+                for key in ("hop1_row_token", "group_offsets", "token_groups", "hop2_src_row"):
+                    assert L[key].tolist() == B[key], key
+
+
+def check_layout_invariants(build_layout, seed=7):
+    rng = np.random.default_rng(seed)
+    T, E, k, R = 400, 32, 6, 8
+    idx, w, er = tiny_routing(seed, T, E, k, R)
+    pp = build_layout(idx, w, er, T // R, R, 0)
+    dd = build_layout(idx, w, er, T // R, R, 1)
+    assert int(pp["num_rows"]) == T * k                       # per-pick: exactly T*k rows
+    dsets = [len({int(er[e]) for e in idx[t]}) for t in range(T)]
+    assert int(dd["num_rows"]) == sum(dsets) <= T * k         # dedup: sum of |D_t|
+    for L in (pp, dd):
+        off = L["rank_offsets"]
+        for d in range(R):                                     # stable: tokens ascending per rank
+            seg = L["row_token"][off[d]:off[d + 1]].astype(np.int64)
+            if L is pp:                                        # per-pick: (expert, token) ascending
+                seg = L["row_expert"][off[d]:off[d + 1]].astype(np.int64) * T + seg
+            assert np.all(np.diff(seg) >= 1)
+        sc = L["send_counts"]
+        assert int(sc.sum()) == int(L["num_rows"])
+        assert np.array_equal(sc.sum(axis=0), np.diff(off))
+    # dedup coefficients add up to each token's total gate weight
+    tot = np.zeros(T)
+    np.add.at(tot, dd["row_token"], dd["row_coef"])
+    np.testing.assert_allclose(tot, w.sum(axis=1), rtol=1e-12)
+    del rng
+
+
+# -------------------------------------------------------------- combine ----
+def check_combine(combine, build_layout, seed=8):
+    rng = np.random.default_rng(seed)
+    T, E, k, R, H = 40, 16, 4, 4, 24
+    idx, w, er = tiny_routing(seed, T, E, k, R)
+    x = rng.standard_normal((T, H))
+    for mode in (0, 1):
+        L = build_layout(idx, w, er, T // R, R, mode)
+        y = x[L["row_token"]]
+        n = int(L["num_rows"])
+        # brute force, ascending rows
+        coef = rng.uniform(-1, 1, size=n)
+        ref = np.zeros((T, H))
+        for t in range(T):
+            for i in range(n):
+                if L["row_token"][i] == t:
+                    ref[t] += coef[i] * y[i]
+        np.testing.assert_allclose(combine(y, L["token_rows"], coef), ref, rtol=1e-12, atol=1e-14)
+        # conservation: coefficient 1 on each token's first row, 0 elsewhere -> X
+        c01 = np.zeros(n)
+        c01[L["token_rows"][:, 0]] = 1.0
+        assert np.array_equal(combine(y, L["token_rows"], c01), x)
+        # all ones -> d_t * X
+        d = (L["token_rows"] >= 0).sum(axis=1)
+        assert np.array_equal(combine(y, L["token_rows"], np.ones(n)), d[:, None] * x)
+        # with the layout's own coefficients and identity experts -> (sum of gate weights) * X
+        np.testing.assert_allclose(combine(y, L["token_rows"], L["row_coef"]),
+                                   w.sum(axis=1)[:, None] * x, rtol=1e-12, atol=1e-14)
+
+
+def check_combine_two_hop(combine_two_hop, build_layout, round_to, seed=9):
+    rng = np.random.default_rng(seed)
+    T, E, k, R, rpg, H = 30, 16, 5, 8, 4, 16
+    idx, w, er = tiny_routing(seed, T, E, k, R)
+    L = build_layout(idx, w, er, -(-T // R), R, 2, ranks_per_group=rpg)
+    n = int(L["num_rows"])
+    y2 = rng.standard_normal((n, H))
+    coef = rng.uniform(0.05, 1, size=n)
+    out, zs = combine_two_hop(y2, L, coef, "bf16")
+    # brute force: group partials per (group, token), rounded, then summed
+    ref = np.zeros((T, H))
+    for t in range(T):
+        groups = sorted({int(er[e]) // rpg for e in idx[t]})
+        for g in groups:
+            z = np.zeros(H)
+            for i in range(n):
+                if L["row_token"][i] == t and L["row_dst"][i] // rpg == g:
+                    z += coef[i] * y2[i]
+            ref[t] += round_to(z, "bf16")
+    np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-15)
+    assert len(zs) == int(L["num_rows_hop1"])
+    # with one rank per group the two hops reduce to the one-hop combine
+    L1 = build_layout(idx, w, er, -(-T // R), R, 2, ranks_per_group=1)
+    x = rng.standard_normal((T, H))
+    y = x[L1["row_token"]]
+    ones = np.ones(int(L1["num_rows"]))
+    out1, _ = combine_two_hop(y, L1, ones, "f32")
+    d = (L1["token_rows"] >= 0).sum(axis=1)
+    np.testing.assert_allclose(out1, d[:, None] * round_to(x, "f32"), rtol=1e-15)
+
+
+# ------------------------------------------------------------- rounding ----
+def check_round_to(round_to):
+    import torch
+    rng = np.random.default_rng(10)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-9, 5, 20000),
+                        rng.standard_normal(2000) * 1e-6,       # f16 subnormals
+                        [0.0, -0.0, 1.0, 65504.0, 6.1e-5]])
+    assert np.array_equal(round_to(x, "f16"), x.astype(np.float16).astype(np.float64))
+    assert np.array_equal(round_to(x, "f32"), x.astype(np.float32).astype(np.float64))
+    xf = x.astype(np.float32)       # f32-exact values: torch's f32 -> bf16 is round-to-nearest-even
+    ref = torch.from_numpy(xf).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(round_to(xf.astype(np.float64), "bf16"), ref)
+    # ties to even
+    assert round_to(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8]), "bf16").tolist() == [1.0, 1 + 2.0 ** -6]

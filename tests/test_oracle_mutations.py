@@ -1,0 +1,147 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and check that
+the pins catch every one of them.  This is what makes the pins worth trusting:
+a dropped term, a wrong sign or index, or a flipped tie rule fails a pin."""
+import numpy as np
+import pytest
+
+import oracle
+import pins
+
+
+def _route_ascending(logits, k, n_groups=0, groups_per_token=0, renormalize=False):
+    idx, w = oracle.route_topk(-np.asarray(logits, np.float32), k, n_groups, groups_per_token, renormalize)
+    p = oracle.softmax(logits)
+    return idx, np.take_along_axis(p, idx.astype(np.int64), 1)
+
+
+def _route_high_tie(logits, k, n_groups=0, groups_per_token=0, renormalize=False):
+    lg = np.asarray(logits, np.float32)[:, ::-1]
+    idx, w = oracle.route_topk(lg, k, n_groups, groups_per_token, renormalize)
+    idx = (lg.shape[1] - 1 - idx).astype(np.int32)
+    p = oracle.softmax(logits)
+    return idx, np.take_along_axis(p, idx.astype(np.int64), 1)
+
+
+def _route_topk_softmax(logits, k, n_groups=0, groups_per_token=0, renormalize=False):
+    # softmax over the k picks only (a dropped normalisation term)
+    idx, w = oracle.route_topk(logits, k, n_groups, groups_per_token, True)
+    return idx, w
+
+
+def _route_group_sum(logits, k, n_groups=0, groups_per_token=0, renormalize=False):
+    lg = np.asarray(logits, np.float32)
+    T, E = lg.shape
+    if not (groups_per_token and groups_per_token < n_groups):
+        return oracle.route_topk(lg, k)
+    gs = E // n_groups
+    score = lg.astype(np.float64).reshape(T, n_groups, gs).sum(axis=2)
+    keep = np.zeros((T, n_groups), bool)
+    np.put_along_axis(keep, np.argsort(-score, axis=1, kind="stable")[:, :groups_per_token], True, axis=1)
+    cand = np.where(np.repeat(keep, gs, axis=1), lg, -np.inf)
+    idx = np.argsort(-cand, axis=1, kind="stable")[:, :k].astype(np.int32)
+    return idx, np.take_along_axis(oracle.softmax(lg), idx.astype(np.int64), 1)
+
+
+@pytest.mark.parametrize("mutant", [_route_ascending, _route_high_tie, _route_topk_softmax])
+def test_route_mutants_caught(mutant):
+    with pytest.raises(AssertionError):
+        pins.check_route_brute(mutant)
+        pins.check_route_special(mutant)
+
+
+def test_group_score_by_sum_caught():
+    with pytest.raises(AssertionError):
+        pins.check_route_groups(_route_group_sum)
+
+
+def _assign_high_rank_tie(counts, off, slots, sr, R):
+    # ties on the activated count go to the HIGHER rank
+    E = len(counts)
+    act = np.zeros(R, np.int64)
+    es, er = np.full(E, -1, np.int32), np.full(E, -1, np.int32)
+    for e in range(E):
+        if counts[e]:
+            s = min(slots[off[e]:off[e + 1]], key=lambda s: (act[sr[s]], -sr[s], s))
+            es[e], er[e] = s, sr[s]
+            act[sr[s]] += 1
+    return es, er, act
+
+
+def _assign_token_count(counts, off, slots, sr, R):
+    # balance demand (token counts) instead of activated experts
+    E = len(counts)
+    load = np.zeros(R, np.int64)
+    act = np.zeros(R, np.int64)
+    es, er = np.full(E, -1, np.int32), np.full(E, -1, np.int32)
+    for e in range(E):
+        if counts[e]:
+            s = min(slots[off[e]:off[e + 1]], key=lambda s: (load[sr[s]], sr[s], s))
+            es[e], er[e] = s, sr[s]
+            load[sr[s]] += counts[e]
+            act[sr[s]] += 1
+    return es, er, act
+
+
+@pytest.mark.parametrize("mutant", [_assign_high_rank_tie, _assign_token_count])
+def test_assign_mutants_caught(mutant):
+    with pytest.raises(AssertionError):
+        pins.check_assign_hand(mutant)
+
+
+def _layout_unstable(idx, w, er, tpr, R, mode, ranks_per_group=0):
+    L = oracle.build_layout(idx, w, er, tpr, R, mode, ranks_per_group)
+    L = dict(L)
+    off = L["rank_offsets"]
+    rt = L["row_token"].copy()
+    for d in range(R):                     # reverse each destination segment
+        rt[off[d]:off[d + 1]] = rt[off[d]:off[d + 1]][::-1]
+    L["row_token"] = rt
+    return L
+
+
+def _layout_no_dedup(idx, w, er, tpr, R, mode, ranks_per_group=0):
+    return oracle.build_layout(idx, w, er, tpr, R, 0 if mode == 1 else mode, ranks_per_group)
+
+
+@pytest.mark.parametrize("mutant", [_layout_unstable, _layout_no_dedup])
+def test_layout_mutants_caught(mutant):
+    with pytest.raises(AssertionError):
+        pins.check_layout_brute(mutant)
+
+
+def _combine_drop_last(y, token_rows, coef, tokens=None):
+    tr = np.asarray(token_rows).copy()
+    last = (tr >= 0).sum(axis=1) - 1
+    tr[np.arange(tr.shape[0]), last] = -1
+    return oracle.combine(y, tr, coef, tokens)
+
+
+def _combine_transposed(y, token_rows, coef, tokens=None):
+    # coefficient of the token instead of the row (an index mix-up)
+    tr = np.asarray(token_rows)
+    c = np.asarray(coef, np.float64)
+    c2 = c[np.minimum(np.arange(c.shape[0]), tr.shape[0] - 1)]
+    return oracle.combine(y, tr, c2, tokens)
+
+
+@pytest.mark.parametrize("mutant", [_combine_drop_last, _combine_transposed])
+def test_combine_mutants_caught(mutant):
+    with pytest.raises(AssertionError):
+        pins.check_combine(mutant, oracle.build_layout)
+
+
+def test_two_hop_without_wire_rounding_caught():
+    def mutant(y2, L, coef, wire_fmt, tokens=None):
+        return oracle.combine_two_hop(y2, L, coef, "f32" if wire_fmt == "bf16" else wire_fmt, tokens)
+    with pytest.raises(AssertionError):
+        pins.check_combine_two_hop(mutant, oracle.build_layout, oracle.round_to)
+
+
+def test_round_half_away_caught():
+    def mutant(x, fmt):
+        r = oracle.round_to(x, fmt)
+        q = oracle.ulp(x, fmt)
+        tie = np.abs(np.abs(np.asarray(x, np.float64) - r) - q / 2) == 0
+        return np.where(tie, np.sign(x) * (np.abs(r) + q * (np.abs(r) < np.abs(x))), r)
+    with pytest.raises(AssertionError):
+        pins.check_round_to(mutant)

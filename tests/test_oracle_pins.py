@@ -1,0 +1,79 @@
+"""The CPU oracle against its pins (no GPU)."""
+import numpy as np
+import pytest
+
+import oracle
+import pins
+
+
+def test_round_to_matches_library_casts():
+    pins.check_round_to(oracle.round_to)
+
+
+def test_route_brute_force_with_ties():
+    pins.check_route_brute(oracle.route_topk)
+
+
+def test_route_library_topk_softmax():
+    pins.check_route_library(oracle.route_topk)
+
+
+def test_route_special_cases():
+    pins.check_route_special(oracle.route_topk)
+
+
+def test_route_group_limited():
+    pins.check_route_groups(oracle.route_topk)
+
+
+def test_hist_counter():
+    pins.check_hist(oracle.demand_hist)
+
+
+def test_assign_hand_worked():
+    pins.check_assign_hand(oracle.replica_assign)
+
+
+def test_assign_page_toy_example():
+    pins.check_assign_toy(oracle.replica_assign, oracle.token_balanced_active)
+
+
+def test_assign_closed_forms():
+    pins.check_assign_closed_forms(oracle.replica_assign)
+
+
+def test_assign_vs_brute_force_optimum():
+    gap = pins.check_assign_brute(oracle.replica_assign, oracle.optimal_max_active)
+    # context, not a bound: the page's greedy was within 10.9% of the optimum on its workload
+    assert 0.0 <= gap < 1.0
+
+
+def test_layout_brute_force_all_modes():
+    pins.check_layout_brute(oracle.build_layout)
+
+
+def test_layout_invariants():
+    pins.check_layout_invariants(oracle.build_layout)
+
+
+def test_combine_brute_and_conservation():
+    pins.check_combine(oracle.combine, oracle.build_layout)
+
+
+def test_combine_two_hop_brute():
+    pins.check_combine_two_hop(oracle.combine_two_hop, oracle.build_layout, oracle.round_to)
+
+
+def test_pack_is_row_gather():
+    rng = np.random.default_rng(0)
+    x = rng.integers(0, 2 ** 16, size=(9, 5), dtype=np.uint16)
+    rt = np.array([3, 3, 0, 8, 1], np.int32)
+    p = oracle.pack(x, rt)
+    for i, t in enumerate(rt):
+        assert p[i].tobytes() == x[t].tobytes()
+    assert oracle.pack(x, rt, rows=[4, 0]).tolist() == [x[1].tolist(), x[3].tolist()]
+
+
+def test_ulp():
+    assert oracle.ulp(np.array([1.0, 1.5, 2.0]), "bf16").tolist() == [2.0 ** -7, 2.0 ** -7, 2.0 ** -6]
+    assert oracle.ulp(np.array([1e-7]), "f16").tolist() == [2.0 ** -24]
