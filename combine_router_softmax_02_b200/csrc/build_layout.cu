@@ -1,0 +1,520 @@
+// Stable per-destination row layout: count kernel + decoupled-lookback scan.
+//
+// Rows are the destination chunks of an AllToAll(-v) ("METRO AllGather vs
+// AllToAll for MoE decode" (fanout.sh), sections "Work the 8-GPU payload
+// example" and "Distinguish METRO from backend names"):
+//   PER_PICK  one row per (token, pick), ordered (rank, expert, token);
+//   DEDUP     one row per (rank, token) in the token's destination set, the
+//             single-send dispatcher of the arXiv:2610.09372 summary
+//             (ainewsletter), section "Two locality techniques";
+//   TWO_HOP   hop-1 rows (group, token) and hop-2 rows (rank, token), the
+//             two-hop dispatch of the TerraceMoE editorial, "The core problem".
+//
+// "Bins" are the segments of the layout: ranks (DEDUP), experts (PER_PICK) or
+// ranks followed by groups (TWO_HOP).  A row's id is
+//   seg_off[bin] + (rows of bin in earlier tiles) + (rows of bin in earlier
+//   warps of the tile) + (rows of bin in earlier lanes of the warp).
+// Kernel 1 (count) builds the per-bin totals with block histograms and global
+// atomics; its last block turns them into segment offsets.  Kernel 2 (place)
+// takes tiles in ticket order, publishes each tile's per-bin aggregate, looks
+// back over its predecessors for the exclusive prefix (bounded waits), and
+// writes the rows.  Within a warp, each lane's distinct bins are merged in
+// ascending key order with redux.sync.min + ballot, which yields both the
+// per-bin counts and each lane's position in token order (stability).
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTile = 256;  // tokens per tile, one per thread
+constexpr int kWarps = kTile / 32;
+constexpr int kMaxBins = kMaxE;  // >= max(E, R + G)
+constexpr int kSendSmem = kMaxR * kMaxR;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr unsigned long long kFlagAgg = 1ull << 32;
+constexpr unsigned long long kFlagInc = 2ull << 32;
+
+struct LayoutArgs {
+  const int *idx;
+  const float *w;
+  const int *expert_rank;
+  int T, tpr, k, E, R, rpg, G, mode, NB, num_tiles;
+  int *counters;  // [0] place-kernel ticket, [1] count-kernel blocks done
+  int *totals;    // [NB]
+  int *seg_off;   // [NB]
+  unsigned long long *state;  // [num_tiles][NB]: flag << 32 | count
+  moe_layout L;
+};
+
+// One token's picks as seen by one thread.
+template <int KM>
+struct TokenPicks {
+  int e[KM];
+  int r[KM];
+  float w[KM];
+  uint32_t present;      // picks with a valid expert and rank
+  unsigned long long dmask;  // ranks of the token
+};
+
+template <int KM>
+__device__ __forceinline__ void load_picks(const LayoutArgs &a, const int *s_er, int t,
+                                           bool want_w, TokenPicks<KM> &p, bool &bad) {
+  p.present = 0;
+  p.dmask = 0;
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    p.e[j] = 0;
+    p.r[j] = 0;
+    p.w[j] = 0.0f;
+    if (j < a.k && t < a.T) {
+      const int e = a.idx[(size_t)t * a.k + j];
+      if ((unsigned)e < (unsigned)a.E) {
+        const int r = s_er[e];
+        if ((unsigned)r < (unsigned)a.R) {
+          p.e[j] = e;
+          p.r[j] = r;
+          p.present |= 1u << j;
+          p.dmask |= 1ull << r;
+          if (want_w) p.w[j] = a.w[(size_t)t * a.k + j];
+        } else {
+          bad = true;
+        }
+      } else {
+        bad = true;
+      }
+    }
+  }
+}
+
+enum Pass { kPassRank = 0, kPassGroup = 1, kPassPick = 2 };
+
+template <int KM>
+__device__ __forceinline__ uint32_t pick_key(const TokenPicks<KM> &p, int j, int pass, int rpg) {
+  if (pass == kPassRank) return (uint32_t)p.r[j];
+  if (pass == kPassGroup) return (uint32_t)(p.r[j] / rpg);
+  return ((uint32_t)p.r[j] << 10) | (uint32_t)p.e[j];
+}
+
+template <int pass>
+__device__ __forceinline__ int key_bin(uint32_t key, int R) {
+  if (pass == kPassRank) return (int)key;
+  if (pass == kPassGroup) return R + (int)key;
+  return (int)(key & 1023u);
+}
+
+// Merge the lanes' distinct keys in ascending order.  For every key present
+// in the warp, f(key, has, ball, c, matched) runs on all lanes: `has` says
+// whether this lane's token has the key, `ball` which lanes do, `c` how many
+// distinct keys this lane had before, `matched` its picks with the key.
+template <int KM, int pass, class F>
+__device__ __forceinline__ void warp_merge(const TokenPicks<KM> &p, int rpg, F &&f) {
+  uint32_t key[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) key[j] = pick_key(p, j, pass, rpg);
+  uint32_t rem = p.present;
+  int c = 0;
+  while (true) {
+    uint32_t mine = 0xffffffffu;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (rem >> j & 1u) mine = min(mine, key[j]);
+    const uint32_t b = __reduce_min_sync(kFull, mine);
+    if (b == 0xffffffffu) break;
+    const bool has = (mine == b);
+    const unsigned ball = __ballot_sync(kFull, has);
+    uint32_t matched = 0;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if ((rem >> j & 1u) && key[j] == b) matched |= 1u << j;
+    f(b, has, ball, c, matched);
+    if (has) {
+      rem &= ~matched;
+      ++c;
+    }
+  }
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ unsigned long long group_bits(int g, int rpg) {
+  const unsigned long long ones = (rpg >= 64) ? ~0ull : ((1ull << rpg) - 1ull);
+  return (rpg >= 64) ? ones : (ones << (g * rpg));
+}
+
+// ------------------------------------------------------------- finalize ----
+// Runs in the last count block: segment offsets and the host-visible offsets.
+__device__ void finalize(const LayoutArgs &a, const int *s_er, DeviceCtx ctx) {
+  if (threadIdx.x != 0) return;
+  const moe_layout &L = a.L;
+  if (a.mode == MOE_LAYOUT_PER_PICK) {
+    int base[kMaxR + 1];
+    for (int r = 0; r <= a.R; ++r) base[r] = 0;
+    for (int e = 0; e < a.E; ++e) {
+      const int r = s_er[e];
+      if ((unsigned)r < (unsigned)a.R) base[r + 1] += __ldcg(a.totals + e);
+    }
+    for (int r = 0; r < a.R; ++r) base[r + 1] += base[r];
+    for (int r = 0; r <= a.R; ++r) L.rank_offsets[r] = base[r];
+    for (int e = 0; e < a.E; ++e) {
+      const int r = s_er[e];
+      if ((unsigned)r < (unsigned)a.R) {
+        a.seg_off[e] = base[r];
+        base[r] += __ldcg(a.totals + e);
+      } else {
+        a.seg_off[e] = 0;
+      }
+    }
+    const int n = L.rank_offsets[a.R];
+    *L.num_rows = n;
+    if (n > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
+    return;
+  }
+  int run = 0;
+  for (int r = 0; r < a.R; ++r) {
+    a.seg_off[r] = run;
+    L.rank_offsets[r] = run;
+    run += __ldcg(a.totals + r);
+  }
+  L.rank_offsets[a.R] = run;
+  *L.num_rows = run;
+  if (run > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
+  if (a.mode == MOE_LAYOUT_TWO_HOP) {
+    int run1 = 0;
+    for (int g = 0; g < a.G; ++g) {
+      a.seg_off[a.R + g] = run1;
+      L.group_offsets[g] = run1;
+      run1 += __ldcg(a.totals + a.R + g);
+    }
+    L.group_offsets[a.G] = run1;
+    *L.num_rows_hop1 = run1;
+    if (run1 > L.capacity_hop1) set_status(ctx.status, MOE_ERR_CAPACITY);
+  }
+}
+
+// ---------------------------------------------------------------- count ----
+template <int KM>
+__global__ void __launch_bounds__(kTile) layout_count_kernel(LayoutArgs a, DeviceCtx ctx) {
+  __shared__ int s_er[kMaxE];
+  __shared__ int s_cnt[kMaxBins];
+  __shared__ int s_send[kSendSmem];
+  __shared__ int s_last;
+  const int tile = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int t = tile * kTile + tid;
+  for (int i = tid; i < a.E; i += kTile) s_er[i] = a.expert_rank[i];
+  for (int i = tid; i < a.NB; i += kTile) {
+    s_cnt[i] = 0;
+    a.state[(size_t)tile * a.NB + i] = 0ull;  // the place kernel's flags start clear
+  }
+  // source ranks are < R, so the block's send-count matrix fits R*R <= 4096 entries
+  for (int i = tid; i < a.R * a.R; i += kTile) s_send[i] = 0;
+  __syncthreads();
+
+  TokenPicks<KM> p;
+  bool bad = false;
+  load_picks<KM>(a, s_er, t, false, p, bad);
+  if (a.mode == MOE_LAYOUT_PER_PICK) {  // the row order needs distinct experts per token
+#pragma unroll
+    for (int i = 0; i < KM; ++i)
+#pragma unroll
+      for (int j = i + 1; j < KM; ++j)
+        if ((p.present >> i & 1u) && (p.present >> j & 1u) && p.e[i] == p.e[j]) {
+          bad = true;
+          p.present &= ~(1u << j);
+        }
+  }
+  const int src = (t < a.T) ? t / a.tpr : 0;
+
+  auto count_send = [&](int dst, bool has, unsigned ball) {
+    if (!has) return;
+    const unsigned peers = __match_any_sync(ball, src);
+    if (lane == __ffs(peers) - 1) atomicAdd(&s_send[src * a.R + dst], __popc(peers));
+  };
+  if (a.mode == MOE_LAYOUT_PER_PICK) {
+    warp_merge<KM, kPassPick>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int, uint32_t) {
+      if (lane == 0) atomicAdd(&s_cnt[key_bin<kPassPick>(b, a.R)], __popc(ball));
+      count_send((int)(b >> 10), has, ball);
+    });
+  } else {
+    warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int, uint32_t) {
+      if (lane == 0) atomicAdd(&s_cnt[key_bin<kPassRank>(b, a.R)], __popc(ball));
+      count_send((int)b, has, ball);
+    });
+    if (a.mode == MOE_LAYOUT_TWO_HOP) {
+      warp_merge<KM, kPassGroup>(p, a.rpg, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
+        if (lane == 0) atomicAdd(&s_cnt[key_bin<kPassGroup>(b, a.R)], __popc(ball));
+      });
+    }
+  }
+  if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
+  __syncthreads();
+  for (int i = tid; i < a.NB; i += kTile)
+    if (s_cnt[i]) atomicAdd(&a.totals[i], s_cnt[i]);
+  for (int i = tid; i < a.R * a.R; i += kTile)
+    if (s_send[i]) atomicAdd(&a.L.send_counts[i], s_send[i]);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&a.counters[1], 1) == a.num_tiles - 1);
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    finalize(a, s_er, ctx);
+  }
+}
+
+// ---------------------------------------------------------------- place ----
+__device__ __forceinline__ unsigned long long wait_published(const unsigned long long *word,
+                                                             const DeviceCtx &ctx, bool &timed_out) {
+  unsigned long long v = ld_acquire_u64(word);
+  if (v >> 32) return v;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    __nanosleep(64);
+    v = ld_acquire_u64(word);
+    if (v >> 32) return v;
+    if (global_ns() - t0 > ctx.wait_limit_ns || ld_volatile_i32(ctx.status) == MOE_ERR_TIMEOUT) {
+      timed_out = true;
+      return kFlagInc;  // treat as an inclusive zero so the chain ends
+    }
+  }
+}
+
+template <int KM>
+__global__ void __launch_bounds__(kTile) layout_place_kernel(LayoutArgs a, DeviceCtx ctx) {
+  __shared__ int s_er[kMaxE];
+  __shared__ int s_wcnt[kWarps][kMaxBins];
+  __shared__ int s_base[kMaxBins];
+  __shared__ int s_tile;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_tile = atomicAdd(&a.counters[0], 1);
+  for (int i = tid; i < a.E; i += kTile) s_er[i] = a.expert_rank[i];
+  for (int i = tid; i < a.NB; i += kTile)
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s_wcnt[w][i] = 0;
+  __syncthreads();
+  const int tile = s_tile;
+  const int t = tile * kTile + tid;
+  const moe_layout &L = a.L;
+
+  TokenPicks<KM> p;
+  bool bad = false;  // reported by the count kernel already
+  load_picks<KM>(a, s_er, t, true, p, bad);
+  if (a.mode == MOE_LAYOUT_PER_PICK) {
+#pragma unroll
+    for (int i = 0; i < KM; ++i)
+#pragma unroll
+      for (int j = i + 1; j < KM; ++j)
+        if ((p.present >> i & 1u) && (p.present >> j & 1u) && p.e[i] == p.e[j]) p.present &= ~(1u << j);
+  }
+
+  // 1. per-warp counts of every bin
+  auto note = [&](int bin, unsigned ball) {
+    if (lane == 0) s_wcnt[warp][bin] = __popc(ball);
+  };
+  if (a.mode == MOE_LAYOUT_PER_PICK) {
+    warp_merge<KM, kPassPick>(p, a.rpg, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
+      note(key_bin<kPassPick>(b, a.R), ball);
+    });
+  } else {
+    warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
+      note(key_bin<kPassRank>(b, a.R), ball);
+    });
+    if (a.mode == MOE_LAYOUT_TWO_HOP)
+      warp_merge<KM, kPassGroup>(p, a.rpg, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
+        note(key_bin<kPassGroup>(b, a.R), ball);
+      });
+  }
+  __syncthreads();
+
+  // 2. tile aggregate, publish, look back, publish the inclusive prefix
+  bool timed_out = false;
+  const bool silent = (tile == ctx.silent_tile);
+  for (int b = tid; b < a.NB; b += kTile) {
+    int agg = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = s_wcnt[w][b];
+      s_wcnt[w][b] = agg;
+      agg += c;
+    }
+    unsigned long long *mine = a.state + (size_t)tile * a.NB + b;
+    int excl = 0;
+    if (tile == 0) {
+      if (!silent) st_release_u64(mine, kFlagInc | (unsigned)agg);
+    } else {
+      if (!silent) st_release_u64(mine, kFlagAgg | (unsigned)agg);
+      for (int q = tile - 1; q >= 0; --q) {
+        const unsigned long long v = wait_published(a.state + (size_t)q * a.NB + b, ctx, timed_out);
+        excl += (int)(unsigned)(v & 0xffffffffull);
+        if ((v >> 32) == 2ull) break;
+      }
+      if (!silent) st_release_u64(mine, kFlagInc | (unsigned)(excl + agg));
+    }
+    s_base[b] = __ldcg(a.seg_off + b) + excl;
+  }
+  if (timed_out) set_status(ctx.status, MOE_ERR_TIMEOUT);
+  __syncthreads();
+
+  // 3. rows (every lane takes part in the merges; lanes past T have no picks)
+  bool over = false;
+  const bool live = t < a.T;
+  const unsigned lt = lanemask_lt();
+  const size_t tk = (size_t)t * a.k;
+  if (a.mode == MOE_LAYOUT_PER_PICK || a.mode == MOE_LAYOUT_DEDUP) {
+    int cnt = 0;
+    auto write_row = [&](int bin, bool has, unsigned ball, int c, uint32_t matched) {
+      if (!has) return;
+      const int row = s_base[bin] + s_wcnt[warp][bin] + __popc(ball & lt);
+      float coef = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (matched >> j & 1u) coef += p.w[j];
+      if (row < L.capacity) {
+        L.row_token[row] = t;
+        L.row_coef[row] = coef;
+        L.token_rows[tk + c] = row;
+      } else {
+        L.token_rows[tk + c] = -1;
+        over = true;
+      }
+      cnt = c + 1;
+    };
+    if (a.mode == MOE_LAYOUT_PER_PICK)
+      warp_merge<KM, kPassPick>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int c, uint32_t m) {
+        write_row(key_bin<kPassPick>(b, a.R), has, ball, c, m);
+      });
+    else
+      warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int c, uint32_t m) {
+        write_row(key_bin<kPassRank>(b, a.R), has, ball, c, m);
+      });
+    if (live)
+      for (int c = cnt; c < a.k; ++c) L.token_rows[tk + c] = -1;
+  } else {
+    // TWO_HOP: hop-1 (group) rows first, then hop-2 (rank) rows
+    unsigned long long gmask = 0;
+    int ng = 0;
+    warp_merge<KM, kPassGroup>(p, a.rpg, [&](uint32_t g, bool has, unsigned ball, int c, uint32_t) {
+      if (!has) return;
+      const int bin = key_bin<kPassGroup>(g, a.R);
+      const int row1 = s_base[bin] + s_wcnt[warp][bin] + __popc(ball & lt);
+      gmask |= 1ull << g;
+      ng = c + 1;
+      if (row1 < L.capacity_hop1) {
+        L.hop1_row_token[row1] = t;
+        L.token_groups[tk + c] = row1;
+        const int nchild = __popcll(p.dmask & group_bits((int)g, a.rpg));
+        for (int ci = nchild; ci < a.k; ++ci) L.hop1_children[(size_t)row1 * a.k + ci] = -1;
+      } else {
+        L.token_groups[tk + c] = -1;
+        over = true;
+      }
+    });
+    if (live)
+      for (int c = ng; c < a.k; ++c) L.token_groups[tk + c] = -1;
+    int nr = 0;
+    warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t r, bool has, unsigned ball, int c, uint32_t matched) {
+      if (!has) return;
+      const int bin = key_bin<kPassRank>(r, a.R);
+      const int row = s_base[bin] + s_wcnt[warp][bin] + __popc(ball & lt);
+      float coef = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (matched >> j & 1u) coef += p.w[j];
+      const int g = (int)r / a.rpg;
+      const int gi = __popcll(gmask & ((1ull << g) - 1ull));
+      const int row1 = L.token_groups[tk + gi];
+      const int ci = __popcll(p.dmask & group_bits(g, a.rpg) & ((1ull << r) - 1ull));
+      nr = c + 1;
+      if (row < L.capacity) {
+        L.row_token[row] = t;
+        L.row_coef[row] = coef;
+        L.token_rows[tk + c] = row;
+        L.hop2_src_row[row] = row1;
+        if (row1 >= 0) L.hop1_children[(size_t)row1 * a.k + ci] = row;
+      } else {
+        L.token_rows[tk + c] = -1;
+        if (row1 >= 0) L.hop1_children[(size_t)row1 * a.k + ci] = -1;
+        over = true;
+      }
+    });
+    if (live)
+      for (int c = nr; c < a.k; ++c) L.token_rows[tk + c] = -1;
+  }
+  if (over) set_status(ctx.status, MOE_ERR_CAPACITY);
+}
+
+template <int KM>
+cudaError_t launch_km(const LayoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+  layout_count_kernel<KM><<<a.num_tiles, kTile, 0, s>>>(a, ctx);
+  cudaError_t err = count_launch(cudaGetLastError());
+  if (err != cudaSuccess) return err;
+  layout_place_kernel<KM><<<a.num_tiles, kTile, 0, s>>>(a, ctx);
+  return count_launch(cudaGetLastError());
+}
+
+int num_bins(int E, int R, int rpg, int mode) {
+  if (mode == MOE_LAYOUT_PER_PICK) return E;
+  if (mode == MOE_LAYOUT_TWO_HOP) return R + R / rpg;
+  return R;
+}
+
+size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+}  // namespace
+
+size_t layout_workspace_bytes(int T, int k, int E, int R, int rpg, int mode) {
+  (void)k;
+  const int NB = num_bins(E, R, rpg, mode);
+  const size_t tiles = (size_t)((T + kTile - 1) / kTile);
+  return align16(sizeof(int) * (2 + 2 * (size_t)NB)) + tiles * NB * sizeof(unsigned long long);
+}
+
+cudaError_t launch_build_layout(const int *idx, const float *w, const int *expert_rank, int T,
+                                int tokens_per_rank, int k, int E, int R, int rpg, int mode,
+                                const moe_layout &L, void *ws, const DeviceCtx &ctx,
+                                cudaStream_t s) {
+  cudaError_t err;
+  if (T == 0) {
+    if ((err = cudaMemsetAsync(L.rank_offsets, 0, sizeof(int) * (R + 1), s)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(L.num_rows, 0, sizeof(int), s)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(L.send_counts, 0, sizeof(int) * R * R, s)) != cudaSuccess) return err;
+    if (mode == MOE_LAYOUT_TWO_HOP) {
+      if ((err = cudaMemsetAsync(L.group_offsets, 0, sizeof(int) * (R / rpg + 1), s)) != cudaSuccess)
+        return err;
+      if ((err = cudaMemsetAsync(L.num_rows_hop1, 0, sizeof(int), s)) != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+  }
+  LayoutArgs a;
+  a.idx = idx;
+  a.w = w;
+  a.expert_rank = expert_rank;
+  a.T = T;
+  a.tpr = tokens_per_rank;
+  a.k = k;
+  a.E = E;
+  a.R = R;
+  a.rpg = (mode == MOE_LAYOUT_TWO_HOP) ? rpg : 1;
+  a.G = (mode == MOE_LAYOUT_TWO_HOP) ? R / rpg : 0;
+  a.mode = mode;
+  a.NB = num_bins(E, R, a.rpg, mode);
+  a.num_tiles = (T + kTile - 1) / kTile;
+  char *base = static_cast<char *>(ws);
+  a.counters = reinterpret_cast<int *>(base);
+  a.totals = a.counters + 2;
+  a.seg_off = a.totals + a.NB;
+  a.state = reinterpret_cast<unsigned long long *>(base + align16(sizeof(int) * (2 + 2 * (size_t)a.NB)));
+  a.L = L;
+  if ((err = cudaMemsetAsync(a.counters, 0, sizeof(int) * (2 + (size_t)a.NB), s)) != cudaSuccess) return err;
+  if ((err = cudaMemsetAsync(L.send_counts, 0, sizeof(int) * (size_t)R * R, s)) != cudaSuccess) return err;
+  if (k <= 2) return launch_km<2>(a, ctx, s);
+  if (k <= 4) return launch_km<4>(a, ctx, s);
+  if (k <= 8) return launch_km<8>(a, ctx, s);
+  return launch_km<16>(a, ctx, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,229 @@
+// Combine: weighted sum of each token's rows back into token order.
+//
+// The combine after the experts ("METRO AllGather vs AllToAll for MoE decode"
+// (fanout.sh), section "changes the routing information"): out[t] = sum over
+// t's rows i, in ascending row order, of coef[i] * y[i], accumulated in
+// float32 and rounded to nearest-even into the output dtype.
+//
+// Generic fan-in, one warp per output row: the item's (<= k) source rows and
+// coefficients are broadcast from lanes 0..k-1, then each lane walks 16-byte
+// column vectors with all of the item's rows in flight at once
+// (ld.global.nc.L1::no_allocate), multiply-adds them in row order and writes
+// the result once.  No atomics: the result does not depend on scheduling.
+//   one-hop:        items = tokens, lists = token_rows
+//   TWO_HOP hop 2:  items = hop-1 rows, lists = hop1_children, output = the
+//                   hop-1 buffer in the activation dtype (the group partial)
+//   TWO_HOP hop 1:  items = tokens, lists = token_groups, coefficients 1
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+struct FaninArgs {
+  const uint8_t *y;
+  uint32_t rb_in;           // input row bytes
+  uint8_t *out;
+  uint32_t rb_out;          // output row bytes
+  int n_items;              // >= 0: item count; < 0: read *n_items_dev
+  const int *n_items_dev;
+  int cap_items;
+  const int *lists;         // [items][k]
+  int k;
+  const float *coef;        // per source row; nullptr = 1
+  int src_cap;              // rows in y
+  int nvec;                 // 16-byte input vectors per row
+};
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+  static constexpr int kPerVec = 4;
+  __device__ static float get(const uint4 &v, int i) { return __uint_as_float((&v.x)[i]); }
+};
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int kPerVec = 8;
+  __device__ static float get(const uint4 &v, int i) {
+    const uint32_t w = (&v.x)[i >> 1];
+    return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+};
+template <>
+struct Elem<__half> {
+  static constexpr int kPerVec = 8;
+  __device__ static float get(const uint4 &v, int i) {
+    const uint32_t w = (&v.x)[i >> 1];
+    return __half2float(__ushort_as_half((unsigned short)((i & 1) ? (w >> 16) : (w & 0xffffu))));
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ uint32_t to_bits16(float f);
+template <>
+__device__ __forceinline__ uint32_t to_bits16<__nv_bfloat16>(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+template <>
+__device__ __forceinline__ uint32_t to_bits16<__half>(float f) {
+  return __half_as_ushort(__float2half_rn(f));
+}
+
+// Store N floats as Tout at p (N * sizeof(Tout) bytes, aligned to that size).
+template <typename Tout, int N>
+__device__ __forceinline__ void store_out(uint8_t *p, const float (&acc)[N]) {
+  if constexpr (sizeof(Tout) == 4) {
+#pragma unroll
+    for (int c = 0; c < N; c += 4)
+      st_v4(p + c * 4, make_uint4(__float_as_uint(acc[c]), __float_as_uint(acc[c + 1]),
+                                  __float_as_uint(acc[c + 2]), __float_as_uint(acc[c + 3])));
+  } else {
+    uint32_t w[N / 2];
+#pragma unroll
+    for (int c = 0; c < N / 2; ++c)
+      w[c] = to_bits16<Tout>(acc[2 * c]) | (to_bits16<Tout>(acc[2 * c + 1]) << 16);
+    if constexpr (N == 8) {
+      st_v4(p, make_uint4(w[0], w[1], w[2], w[3]));
+    } else {
+      asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(w[0]), "r"(w[1]) : "memory");
+    }
+  }
+}
+
+template <typename Tin, typename Tout, int KM>
+__global__ void __launch_bounds__(256) fanin_kernel(FaninArgs a, DeviceCtx ctx) {
+  constexpr int VE = Elem<Tin>::kPerVec;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  int n = a.n_items;
+  if (n < 0) n = min(max(*a.n_items_dev, 0), a.cap_items);
+  bool bounds = false;
+  for (int item = blockIdx.x * wpb + (threadIdx.x >> 5); item < n; item += gridDim.x * wpb) {
+    int my_r = -1;
+    float my_c = 0.0f;
+    if (lane < a.k) {
+      my_r = __ldcs(a.lists + (size_t)item * a.k + lane);
+      if (my_r >= a.src_cap || my_r < -1) {
+        bounds = true;
+        my_r = -1;
+      }
+      if (my_r >= 0) my_c = a.coef ? __ldg(a.coef + my_r) : 1.0f;
+    }
+    const unsigned vmask = __ballot_sync(kFull, my_r >= 0);
+    int rows[KM];
+    float cf[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      rows[j] = __shfl_sync(kFull, my_r, j);
+      cf[j] = __shfl_sync(kFull, my_c, j);
+    }
+    uint8_t *orow = a.out + (size_t)item * a.rb_out;
+    for (int v = lane; v < a.nvec; v += 32) {
+      uint4 d[KM];
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (vmask >> j & 1u) d[j] = ld_stream_v4(a.y + (size_t)rows[j] * a.rb_in + (size_t)v * 16);
+      float acc[VE];
+#pragma unroll
+      for (int e = 0; e < VE; ++e) acc[e] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (vmask >> j & 1u)
+#pragma unroll
+          for (int e = 0; e < VE; ++e) acc[e] = fmaf(cf[j], Elem<Tin>::get(d[j], e), acc[e]);
+      store_out<Tout, VE>(orow + (size_t)v * VE * sizeof(Tout), acc);
+    }
+  }
+  if (bounds) set_status(ctx.status, MOE_ERR_BOUNDS);
+}
+
+template <typename Tin, typename Tout, int KM>
+cudaError_t launch3(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+  const int wpb = 8;
+  long blocks = (a.n_items >= 0) ? ((long)a.n_items + wpb - 1) / wpb : (long)ctx.num_sms * 8;
+  const long cap = (long)ctx.num_sms * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks <= 0) return cudaSuccess;
+  fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, wpb * 32, 0, s>>>(a, ctx);
+  return count_launch(cudaGetLastError());
+}
+
+template <typename Tin, typename Tout>
+cudaError_t launch2(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+  if (a.k <= 2) return launch3<Tin, Tout, 2>(a, ctx, s);
+  if (a.k <= 4) return launch3<Tin, Tout, 4>(a, ctx, s);
+  if (a.k <= 8) return launch3<Tin, Tout, 8>(a, ctx, s);
+  return launch3<Tin, Tout, 16>(a, ctx, s);
+}
+
+template <typename Tin>
+cudaError_t launch1(const FaninArgs &a, int out_dtype, const DeviceCtx &ctx, cudaStream_t s) {
+  if (out_dtype == MOE_F16) return launch2<Tin, __half>(a, ctx, s);
+  if (out_dtype == MOE_BF16) return launch2<Tin, __nv_bfloat16>(a, ctx, s);
+  return launch2<Tin, float>(a, ctx, s);
+}
+
+cudaError_t launch_fanin(const FaninArgs &a, int in_dtype, int out_dtype, const DeviceCtx &ctx,
+                         cudaStream_t s) {
+  if (a.n_items == 0) return cudaSuccess;
+  if (in_dtype == MOE_F16) return launch1<__half>(a, out_dtype, ctx, s);
+  if (in_dtype == MOE_BF16) return launch1<__nv_bfloat16>(a, out_dtype, ctx, s);
+  return launch1<float>(a, out_dtype, ctx, s);
+}
+
+int elem_size(int dt) { return dt == MOE_F32 ? 4 : 2; }
+
+}  // namespace
+
+cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
+                           const float *row_coef, void *out, int out_dtype, void *hop1_buf,
+                           const DeviceCtx &ctx, cudaStream_t s) {
+  const float *coef = row_coef ? row_coef : L.row_coef;
+  FaninArgs a;
+  a.k = L.k;
+  a.n_items_dev = nullptr;
+  a.cap_items = 0;
+  if (L.mode != MOE_LAYOUT_TWO_HOP) {
+    a.y = static_cast<const uint8_t *>(y);
+    a.rb_in = (uint32_t)((size_t)H * elem_size(dtype));
+    a.out = static_cast<uint8_t *>(out);
+    a.rb_out = (uint32_t)((size_t)H * elem_size(out_dtype));
+    a.n_items = L.T;
+    a.lists = L.token_rows;
+    a.coef = coef;
+    a.src_cap = L.capacity;
+    a.nvec = (int)(a.rb_in / 16);
+    return launch_fanin(a, dtype, out_dtype, ctx, s);
+  }
+  // hop 2 reverse: rank rows -> group partials in the activation dtype
+  a.y = static_cast<const uint8_t *>(y);
+  a.rb_in = (uint32_t)((size_t)H * elem_size(dtype));
+  a.out = static_cast<uint8_t *>(hop1_buf);
+  a.rb_out = a.rb_in;
+  a.n_items = -1;
+  a.n_items_dev = L.num_rows_hop1;
+  a.cap_items = L.capacity_hop1;
+  a.lists = L.hop1_children;
+  a.coef = coef;
+  a.src_cap = L.capacity;
+  a.nvec = (int)(a.rb_in / 16);
+  cudaError_t err = launch_fanin(a, dtype, dtype, ctx, s);
+  if (err != cudaSuccess) return err;
+  // hop 1 reverse: group partials -> token
+  a.y = static_cast<const uint8_t *>(hop1_buf);
+  a.out = static_cast<uint8_t *>(out);
+  a.rb_out = (uint32_t)((size_t)H * elem_size(out_dtype));
+  a.n_items = L.T;
+  a.n_items_dev = nullptr;
+  a.lists = L.token_groups;
+  a.coef = nullptr;
+  a.src_cap = L.capacity_hop1;
+  return launch_fanin(a, dtype, out_dtype, ctx, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,205 @@
+// Internal declarations shared by the kernels of libmoe.so (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/moe.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libmoe targets sm_100a only"
+#endif
+
+namespace moe {
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 16;
+constexpr int kMaxR = 64;
+constexpr int kMaxGroups = 32;
+constexpr int kMaxSlots = 32768;
+
+// Settings every launch receives by value.
+struct DeviceCtx {
+  int *status;            // per-device status word (first error wins)
+  uint64_t wait_limit_ns; // limit of every bounded wait
+  int silent_tile;        // layout scan tile that does not publish (-1: none)
+  int num_sms;
+};
+
+// ---------------------------------------------------------------- device ----
+__device__ __forceinline__ void set_status(int *status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ int ld_volatile_i32(const int *p) {
+  int v;
+  asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// mbarrier + bulk async copies (TMA without tensor maps), shared::cta forms.
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase; false if the limit ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// global -> shared bulk copy completing on an mbarrier (bytes % 16 == 0, 16-B aligned).
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
+                                         uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_addr(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// shared -> global bulk copy in the thread's bulk async-group.
+__device__ __forceinline__ void bulk_s2g(void *dst_gmem, const void *src_smem, uint32_t bytes,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;"
+      ::"l"(dst_gmem), "r"(smem_addr(src_smem)), "r"(bytes), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 16-byte streaming load (read-only path, no L1 allocation).
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_v4(void *p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+// ------------------------------------------------------------------ host ----
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <class Kern>
+inline cudaError_t set_smem_limit_once(Kern kern, int bytes, std::atomic<unsigned long long> &done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+// Host-side count of kernel launches (moe_kernel_launches); each launch site
+// calls count_launch() after a launch that cudaGetLastError() accepted.
+extern std::atomic<unsigned long long> g_kernel_launches;
+inline cudaError_t count_launch(cudaError_t e) {
+  if (e == cudaSuccess) g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+// Kernel launchers (defined next to their kernels).  Each returns a
+// cudaError_t from cudaGetLastError() after the launch.
+cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int n_groups, int gpt,
+                              int renorm, int *idx, float *w, const DeviceCtx &ctx,
+                              cudaStream_t s);
+cudaError_t launch_demand_hist(const int *idx, int T, int k, int E, int *counts,
+                               const DeviceCtx &ctx, cudaStream_t s);
+cudaError_t launch_replica_assign(const int *counts, int E, const int *off, const int *slots,
+                                  int n_entries, const int *slot_rank, int S, int R,
+                                  int *expert_slot, int *expert_rank, int *rank_active,
+                                  const DeviceCtx &ctx, cudaStream_t s);
+size_t layout_workspace_bytes(int T, int k, int E, int R, int rpg, int mode);
+cudaError_t launch_build_layout(const int *idx, const float *w, const int *expert_rank, int T,
+                                int tokens_per_rank, int k, int E, int R, int rpg, int mode,
+                                const moe_layout &L, void *ws, const DeviceCtx &ctx,
+                                cudaStream_t s);
+cudaError_t launch_pack(const void *x, int elem_bytes, int H, const moe_layout &L, void *packed,
+                        void *packed_hop1, const DeviceCtx &ctx, cudaStream_t s);
+cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
+                           const float *row_coef, void *out, int out_dtype, void *hop1_buf,
+                           const DeviceCtx &ctx, cudaStream_t s);
+
+}  // namespace moe

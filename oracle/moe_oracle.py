@@ -286,6 +286,9 @@ def build_layout(idx: np.ndarray, w: np.ndarray, expert_rank: np.ndarray,
         # hop-2 row (dst, t) reads hop-1 row (dst // rpg, t)
         src_key = (row_dst // rpg) * T + row_token
         out["hop2_src_row"] = np.searchsorted(gkey, src_key).astype(np.int32)
+        # each hop-1 row's hop-2 rows, ascending
+        out["hop1_children"] = _rows_per_token(out["hop2_src_row"].astype(np.int64),
+                                               gkey.shape[0], k).astype(np.int32)
     return out
 
 

@@ -253,6 +253,8 @@ def brute_layout(idx, w, expert_rank, tokens_per_rank, R, mode, rpg=0):
         tg = [[i for i, (g, t2) in enumerate(h1) if t2 == t] for t in range(T)]
         out["token_groups"] = [x + [-1] * (k - len(x)) for x in tg]
         out["hop2_src_row"] = [h1.index((d // rpg, t)) for d, t, _ in rows]
+        ch = [[i for i, s in enumerate(out["hop2_src_row"]) if s == r1] for r1 in range(len(h1))]
+        out["hop1_children"] = [x + [-1] * (k - len(x)) for x in ch]
     return out
 
 
@@ -286,7 +288,7 @@ def check_layout_brute(build_layout):
             assert L["send_counts"].tolist() == B["send_counts"]
             assert int(L["num_rows"]) == len(B["row_token"])
             if mode == 2:
-                for key in ("hop1_row_token", "group_offsets", "token_groups", "hop2_src_row"):
+                for key in ("hop1_row_token", "group_offsets", "token_groups", "hop2_src_row", "hop1_children"):
                     assert L[key].tolist() == B[key], key
 
 

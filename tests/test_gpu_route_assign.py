@@ -1,0 +1,151 @@
+"""GPU parity: router top-k, demand histogram and METRO assignment against the
+CPU oracle, through the C ABI (bit-exact indices and counts, derived bounds
+on the weights)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pins
+import workloads as W
+from gpu_util import assert_weights, moe, to_dev  # noqa: F401
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", sorted(W.CONFIGS))
+def test_route_full_size_configs(moe, name):
+    cfg = W.CONFIGS[name]
+    logits = W.make_logits(cfg, seed=0)
+    idx_d, w_d = moe.route_topk(to_dev(logits), cfg.k, cfg.n_groups, cfg.groups_per_token)
+    assert moe.get_status() == 0
+    idx, w = oracle.route_topk(logits, cfg.k, cfg.n_groups, cfg.groups_per_token)
+    assert np.array_equal(idx_d.cpu().numpy(), idx)
+    assert_weights(w_d.cpu().numpy(), w, logits, idx)
+
+
+@pytest.mark.parametrize("T,E,k,G,gpt,renorm,ties", [
+    (1, 64, 2, 0, 0, 0, False),
+    (33, 40, 3, 0, 0, 0, False),        # E not a multiple of 32, ragged token count
+    (300, 1024, 16, 0, 0, 0, False),    # largest E and k
+    (77, 6, 6, 0, 0, 0, False),         # k = E
+    (64, 1, 1, 0, 0, 0, False),
+    (500, 256, 8, 0, 0, 1, False),      # renormalised weights
+    (1000, 64, 8, 0, 0, 0, True),       # many exact ties
+    (700, 128, 8, 8, 4, 0, False),      # group-limited, the two-hop config's shape
+    (300, 96, 5, 32, 3, 0, True),       # 32 groups of 3, ties
+    (129, 32, 4, 4, 1, 0, True),
+])
+def test_route_edges(moe, T, E, k, G, gpt, renorm, ties):
+    rng = np.random.default_rng(T * 7 + E)
+    if ties:
+        logits = (rng.integers(-2, 3, size=(T, E)) * 0.5).astype(np.float32)
+        logits[::5] = 0.0
+        logits[1::7, ::3] = -0.0            # -0 and +0 tie like the floats compare
+    else:
+        logits = rng.standard_normal((T, E)).astype(np.float32) * 3
+    idx_d, w_d = moe.route_topk(to_dev(logits), k, G, gpt, bool(renorm))
+    assert moe.get_status() == 0
+    idx, w = oracle.route_topk(logits, k, G, gpt, bool(renorm))
+    assert np.array_equal(idx_d.cpu().numpy(), idx)
+    assert_weights(w_d.cpu().numpy(), w, logits, idx, renormalize=bool(renorm))
+
+
+def test_route_group_fixtures(moe):
+    g = pins.golden("p4_group_limited.json")
+    for c in g["cases"]:
+        lg = np.asarray([c["logits"]], np.float32)
+        idx_d, _ = moe.route_topk(to_dev(lg), c["k"], c["n_groups"], c["groups_per_token"])
+        assert idx_d.cpu().numpy()[0].tolist() == c["idx"]
+
+
+def test_route_nonfinite_logit_reported(moe):
+    lg = np.zeros((4, 8), np.float32)
+    lg[2, 3] = np.nan
+    moe.route_topk(to_dev(lg), 2)
+    assert moe.get_status() == 6            # MOE_ERR_BAD_INPUT
+    assert moe.get_status() == 0            # read-and-clear
+
+
+def test_route_zero_tokens(moe):
+    idx, w = moe.route_topk(torch.empty((0, 16), dtype=torch.float32, device="cuda"), 2)
+    assert idx.shape == (0, 2) and moe.get_status() == 0
+
+
+@pytest.mark.parametrize("name", sorted(W.CONFIGS))
+def test_hist_full_size(moe, name):
+    cfg = W.CONFIGS[name]
+    idx, _ = oracle.route_topk(W.make_logits(cfg, 0), cfg.k, cfg.n_groups, cfg.groups_per_token)
+    c_d = moe.demand_hist(to_dev(idx), cfg.E)
+    assert moe.get_status() == 0
+    assert np.array_equal(c_d.cpu().numpy(), oracle.demand_hist(idx, cfg.E))
+
+
+def test_hist_bad_id_and_skew(moe):
+    idx = np.zeros((5000, 4), np.int32)          # every pick on expert 0: worst contention
+    idx[:, 1:] = np.arange(1, 4)
+    idx[17, 2] = 99                               # out of range
+    c_d = moe.demand_hist(to_dev(idx), 8)
+    assert moe.get_status() == 6
+    c = c_d.cpu().numpy()
+    assert c[0] == 5000 and c[2] == 4999 and c.sum() == 5000 * 4 - 1
+
+
+def _assign_dev(moe, counts, rm_off, rm_slots, slot_rank, R):
+    s, r, a = moe.replica_assign(to_dev(np.asarray(counts, np.int32)), to_dev(np.asarray(rm_off, np.int32)),
+                                 to_dev(np.asarray(rm_slots, np.int32)), to_dev(np.asarray(slot_rank, np.int32)), R)
+    return s.cpu().numpy(), r.cpu().numpy(), a.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", sorted(W.CONFIGS))
+def test_assign_configs(moe, name):
+    cfg = W.CONFIGS[name]
+    rm = W.make_replica_map(cfg, 0)
+    idx, _ = oracle.route_topk(W.make_logits(cfg, 0), cfg.k, cfg.n_groups, cfg.groups_per_token)
+    counts = oracle.demand_hist(idx, cfg.E)
+    got = _assign_dev(moe, counts, rm.replica_offsets, rm.replica_slots, rm.slot_rank, cfg.R)
+    assert moe.get_status() == 0
+    ref = oracle.replica_assign(counts, rm.replica_offsets, rm.replica_slots, rm.slot_rank, cfg.R)
+    for g, r in zip(got, ref):
+        assert np.array_equal(g, r.astype(np.int32))
+
+
+def test_assign_hand_worked_and_toy(moe):
+    g = pins.golden("metro_greedy_hand.json")
+    s, r, a = _assign_dev(moe, g["counts"], g["replica_offsets"], g["replica_slots"], g["slot_rank"], g["R"])
+    assert s.tolist() == g["expert_slot"] and r.tolist() == g["expert_rank"]
+    assert a.tolist() == g["rank_active"]
+    gt, counts, off, slots, sr, R = pins.toy_instance()
+    _, _, a = _assign_dev(moe, counts, off, slots, sr, R)
+    assert int(a.max()) == gt["metro_max_active_per_gpu"]
+
+
+def test_assign_random_maps_with_ties(moe):
+    rng = np.random.default_rng(11)
+    for trial in range(40):
+        E, R = int(rng.integers(1, 300)), int(rng.integers(1, 65))
+        nrep = rng.integers(1, min(R, 40) + 1, size=E)   # up to 40 replicas: two lane rounds
+        if trial % 5 == 0:
+            nrep[:] = 1
+        reps = [rng.choice(R, size=int(n), replace=False) for n in nrep]
+        slot_rank = np.concatenate(reps).astype(np.int32)
+        S = slot_rank.shape[0]
+        perm = rng.permutation(S)                        # slot ids not in expert order
+        sr_by_slot = np.empty(S, np.int32)
+        sr_by_slot[perm] = slot_rank
+        off = np.zeros(E + 1, np.int32)
+        off[1:] = np.cumsum(nrep)
+        slots = perm.astype(np.int32)
+        counts = rng.integers(0, 3, size=E).astype(np.int32)
+        got = _assign_dev(moe, counts, off, slots, sr_by_slot, R)
+        assert moe.get_status() == 0
+        ref = oracle.replica_assign(counts, off, slots, sr_by_slot, R)
+        for g, r in zip(got, ref):
+            assert np.array_equal(g, r.astype(np.int32)), trial
+
+
+def test_assign_active_expert_without_replica(moe):
+    counts = [1, 2, 0]
+    s, r, a = _assign_dev(moe, counts, [0, 1, 1, 2], [0, 1], [0, 1], 2)
+    assert moe.get_status() == 6
+    assert s.tolist() == [0, -1, -1] and r.tolist() == [0, -1, -1] and a.tolist() == [1, 0]
