@@ -55,6 +55,8 @@ _SIGS = {
     "moe_layout_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "moe_build_layout": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                         ctypes.POINTER(moe_layout), _P, _SZ, _S]),
+    "moe_build_layout_static": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                               ctypes.POINTER(moe_layout), _S]),
     "moe_pack": (ctypes.c_int, [_P, _I, _I, ctypes.POINTER(moe_layout), _P, _P, _S]),
     "moe_combine": (ctypes.c_int, [_P, _I, _I, ctypes.POINTER(moe_layout), _P, _P, _I, _P, _S]),
     "moe_get_status": (ctypes.c_int, [_S]),

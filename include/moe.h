@@ -185,6 +185,36 @@ MOE_API int moe_build_layout(const int32_t *topk_idx, const float *topk_w, const
                      void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /*
+ * moe_build_layout without a workspace argument.  The paper has no
+ * counterpart: this is a convenience of this library.
+ *
+ * Some callers cannot allocate device memory on the call path -- a serving
+ * loop that reserves all of its memory at start-up and allows no allocation
+ * per request, or a host framework that hands a library only its existing
+ * input and output buffers and exposes no allocator -- so they cannot supply
+ * the scratch workspace moe_build_layout needs.  This variant takes its
+ * scratch from a fixed array of MOE_LAYOUT_STATIC_SCRATCH_BYTES in device
+ * memory that the library reserves when it is loaded (every GPU that loads the
+ * library holds it until the process exits) and calls no allocator.
+ *
+ * Arguments, outputs and device-side errors are those of moe_build_layout.
+ * Returns MOE_ERR_UNSUPPORTED, before anything is launched, when
+ * moe_layout_workspace_size() for these sizes exceeds
+ * MOE_LAYOUT_STATIC_SCRATCH_BYTES (for example 65536 tokens over 64 ranks
+ * needs 131 KB in DEDUP mode).  The first call on a device looks up the
+ * array's device address with that device current; make that first call
+ * before any stream capture.  All calls share the one array, whose contents
+ * persist from call to call (each call clears what must start at zero):
+ * calls whose executions overlap on the GPU -- on different streams, or from
+ * different host threads -- race on it and must be serialised by the caller.
+ */
+#define MOE_LAYOUT_STATIC_SCRATCH_BYTES (1u << 20)
+MOE_API int moe_build_layout_static(const int32_t *topk_idx, const float *topk_w,
+                                    const int32_t *expert_rank, int32_t T, int32_t tokens_per_rank,
+                                    int32_t k, int32_t E, int32_t R, int32_t ranks_per_group,
+                                    int32_t mode, moe_layout *layout, moe_stream_t stream);
+
+/*
  * Pack: packed[row] = x[row_token[row]] for every row (a bit copy), token
  * major: each token row is read once and written to each of its rows.
  * Source: the local half of the AllToAll dispatch ("METRO AllGather vs
