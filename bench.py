@@ -160,7 +160,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    cfg = W.CONFIGS[args.config]
+    cfg = config_of(args)
     seed = args.seed + rank
     logits_h = torch.from_numpy(W.make_logits(cfg, seed)).pin_memory()
     x_h = W.make_activations(cfg, seed).pin_memory()
@@ -365,10 +365,17 @@ def cpu_baseline(cfg: W.Config, args):
             "host_cpus": os.cpu_count()}
 
 
+def config_of(args) -> W.Config:
+    cfg = W.CONFIGS[args.config]
+    if args.tokens:
+        cfg = cfg.with_(T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
+    return cfg
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return None
-    cfg = W.CONFIGS[args.config]
+    cfg = config_of(args)
     tokens = min(cfg.T, args.ref_sample_tokens)
     sub, logits, x32, rm = oracle_sample(cfg, tokens, args.seed)
     for _ in range(args.warmup):
@@ -404,6 +411,8 @@ def main(argv=None):
     ap.add_argument("--config", default="c4", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload with this many tokens instead (profiling captures)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8192)
     ap.add_argument("--ref-sample-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
