@@ -1,0 +1,73 @@
+"""Multi-rank host logic of bench.py on CPU (gloo, world size 2): the timing
+aggregation takes the slowest rank's time and sums the rows of all ranks, and
+under torchrun the reference arm prints one line from rank 0 only."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    times = [10.0 + 5 * rank, 100.0 - rank]
+    rows = [1000 * (rank + 1), 7]
+    t, r = bench.aggregate(dist, "cpu", times, rows)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, t, r))
+
+
+def test_aggregate_max_time_sum_rows_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, t, r in res:
+        assert t == [15.0, 100.0]          # slowest rank per timed region
+        assert r == [3000.0, 14.0]         # rows of all ranks
+
+
+def test_aggregate_single_process_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.aggregate(None, "cpu", [3.0], [5]) == ([3.0], [5])
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+           "--ref-sample-tokens", "128", "--config", "c1"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
