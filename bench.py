@@ -138,9 +138,10 @@ def step_bytes(cfg: W.Config, rows: int, rows_hop1: int, S: int) -> dict:
     }
     if cfg.mode == W.TWO_HOP:
         d["build_layout"] += rows_hop1 * (4 + k * 4) + T * k * 4 + rows * 4
-        d["pack"] = (T + rows_hop1) * H * b + (rows_hop1 + rows) * H * b + T * k * 4 + rows_hop1 * k * 4
-        d["combine"] = (rows + rows_hop1) * H * b + (rows_hop1 + T) * H * b + rows * 4 + \
-            rows_hop1 * k * 4 + T * k * 4
+        # one read of each token, both hops' rows written
+        d["pack"] = (T + rows_hop1 + rows) * H * b + 2 * T * k * 4
+        # rank rows read once; group partials and tokens written
+        d["combine"] = (rows + rows_hop1 + T) * H * b + rows * 8 + T * k * 4
     else:
         d["pack"] = (T + rows) * H * b + T * k * 4
         d["combine"] = (rows + T) * H * b + rows * 4 + T * k * 4

@@ -252,7 +252,9 @@ def pack(x: torch.Tensor, layout: Layout, packed=None, packed_hop1=None, stream=
 
 
 def combine(y: torch.Tensor, layout: Layout, out=None, out_dtype=None, row_coef=None,
-            hop1_buf=None, stream=None):
+            hop1_buf=None, stream=None, store_hop1: bool = True):
+    """TWO_HOP: the group partials go to hop1_buf (allocated if None), or are
+    not stored at all with store_hop1=False."""
     if y.dtype not in _DT:
         raise TypeError("y must be float16, bfloat16 or float32")
     _need(y, y.dtype, "y", 2)
@@ -264,8 +266,10 @@ def combine(y: torch.Tensor, layout: Layout, out=None, out_dtype=None, row_coef=
     _need(out, out_dtype, "out", 2)
     if row_coef is not None:
         _need(row_coef, torch.float32, "row_coef", 1)
-    if L.mode == TWO_HOP and hop1_buf is None:
+    if L.mode == TWO_HOP and hop1_buf is None and store_hop1:
         hop1_buf = torch.empty((max(L.capacity_hop1, 1), H), dtype=y.dtype, device=y.device)
+    if not store_hop1:
+        hop1_buf = None
     _check(lib().moe_combine(_p(y), _DT[y.dtype], H, ctypes.byref(L.struct), _p(row_coef), _p(out),
                              _DT[out_dtype], _p(hop1_buf), _stream(stream)), "moe_combine")
     return out

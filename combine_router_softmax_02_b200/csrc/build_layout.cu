@@ -18,9 +18,12 @@
 // atomics; its last block turns them into segment offsets.  Kernel 2 (place)
 // takes tiles in ticket order, publishes each tile's per-bin aggregate, looks
 // back over its predecessors for the exclusive prefix (bounded waits), and
-// writes the rows.  Within a warp, each lane's distinct bins are merged in
-// ascending key order with redux.sync.min + ballot, which yields both the
-// per-bin counts and each lane's position in token order (stability).
+// writes the rows.  Within a warp a bin's ballot over the lanes gives both its
+// count and each lane's position in token order (stability).  Ranks and
+// groups (at most 64 each) are 64-bit masks per token: one ballot per bin
+// present in the warp, then each lane walks its own bits.  Experts (PER_PICK,
+// up to 1024 bins) are merged instead: each round takes the smallest key
+// (rank << 10 | expert) left in the warp with redux.sync.min.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -54,6 +57,7 @@ struct TokenPicks {
   float w[KM];
   uint32_t present;      // picks with a valid expert and rank
   unsigned long long dmask;  // ranks of the token
+  unsigned long long gmask;  // groups of the token (TWO_HOP)
 };
 
 template <int KM>
@@ -61,6 +65,7 @@ __device__ __forceinline__ void load_picks(const LayoutArgs &a, const int *s_er,
                                            bool want_w, TokenPicks<KM> &p, bool &bad) {
   p.present = 0;
   p.dmask = 0;
+  p.gmask = 0;
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
     p.e[j] = 0;
@@ -75,6 +80,7 @@ __device__ __forceinline__ void load_picks(const LayoutArgs &a, const int *s_er,
           p.r[j] = r;
           p.present |= 1u << j;
           p.dmask |= 1ull << r;
+          p.gmask |= 1ull << (r / a.rpg);
           if (want_w) p.w[j] = a.w[(size_t)t * a.k + j];
         } else {
           bad = true;
@@ -131,6 +137,25 @@ __device__ __forceinline__ void warp_merge(const TokenPicks<KM> &p, int rpg, F &
       rem &= ~matched;
       ++c;
     }
+  }
+}
+
+__device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
+  const unsigned lo = __reduce_or_sync(kFull, (unsigned)m);
+  const unsigned hi = __reduce_or_sync(kFull, (unsigned)(m >> 32));
+  return ((unsigned long long)hi << 32) | lo;
+}
+
+// Bins given as 64-bit masks (ranks, or groups): for every bin present in the
+// warp, f(bin, has, ball) runs on all lanes with the warp's ballot of the bin.
+template <class F>
+__device__ __forceinline__ void warp_mask_bins(unsigned long long mask, F &&f) {
+  unsigned long long wm = warp_or64(mask);
+  while (wm) {
+    const int b = __ffsll((long long)wm) - 1;
+    wm &= wm - 1;
+    const bool has = (mask >> b) & 1ull;
+    f(b, has, __ballot_sync(kFull, has));
   }
 }
 
@@ -227,11 +252,13 @@ __global__ void __launch_bounds__(kTile) layout_count_kernel(LayoutArgs a, Devic
           p.present &= ~(1u << j);
         }
   }
-  const int src = (t < a.T) ? t / a.tpr : 0;
+  const int src0 = __shfl_sync(kFull, (t < a.T) ? t / a.tpr : 0, 0);
+  const int src = (t < a.T) ? t / a.tpr : src0;
+  const bool src_uniform = __all_sync(kFull, src == src0);  // one source rank in the warp
 
   auto count_send = [&](int dst, bool has, unsigned ball) {
     if (!has) return;
-    const unsigned peers = __match_any_sync(ball, src);
+    const unsigned peers = src_uniform ? ball : __match_any_sync(ball, src);
     if (lane == __ffs(peers) - 1) atomicAdd(&s_send[src * a.R + dst], __popc(peers));
   };
   if (a.mode == MOE_LAYOUT_PER_PICK) {
@@ -240,15 +267,14 @@ __global__ void __launch_bounds__(kTile) layout_count_kernel(LayoutArgs a, Devic
       count_send((int)(b >> 10), has, ball);
     });
   } else {
-    warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int, uint32_t) {
-      if (lane == 0) atomicAdd(&s_cnt[key_bin<kPassRank>(b, a.R)], __popc(ball));
-      count_send((int)b, has, ball);
+    warp_mask_bins(p.dmask, [&](int r, bool has, unsigned ball) {
+      if (lane == 0) atomicAdd(&s_cnt[r], __popc(ball));
+      count_send(r, has, ball);
     });
-    if (a.mode == MOE_LAYOUT_TWO_HOP) {
-      warp_merge<KM, kPassGroup>(p, a.rpg, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
-        if (lane == 0) atomicAdd(&s_cnt[key_bin<kPassGroup>(b, a.R)], __popc(ball));
+    if (a.mode == MOE_LAYOUT_TWO_HOP)
+      warp_mask_bins(p.gmask, [&](int g, bool, unsigned ball) {
+        if (lane == 0) atomicAdd(&s_cnt[a.R + g], __popc(ball));
       });
-    }
   }
   if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
   __syncthreads();
@@ -288,6 +314,7 @@ __global__ void __launch_bounds__(kTile) layout_place_kernel(LayoutArgs a, Devic
   __shared__ int s_er[kMaxE];
   __shared__ int s_wcnt[kWarps][kMaxBins];
   __shared__ int s_base[kMaxBins];
+  __shared__ unsigned s_wball[kWarps][2 * kMaxR];  // mask bins: each warp's ballot per bin
   __shared__ int s_tile;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) s_tile = atomicAdd(&a.counters[0], 1);
@@ -320,12 +347,14 @@ __global__ void __launch_bounds__(kTile) layout_place_kernel(LayoutArgs a, Devic
       note(key_bin<kPassPick>(b, a.R), ball);
     });
   } else {
-    warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
-      note(key_bin<kPassRank>(b, a.R), ball);
+    warp_mask_bins(p.dmask, [&](int r, bool, unsigned ball) {
+      note(r, ball);
+      if (lane == 0) s_wball[warp][r] = ball;
     });
     if (a.mode == MOE_LAYOUT_TWO_HOP)
-      warp_merge<KM, kPassGroup>(p, a.rpg, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
-        note(key_bin<kPassGroup>(b, a.R), ball);
+      warp_mask_bins(p.gmask, [&](int g, bool, unsigned ball) {
+        note(a.R + g, ball);
+        if (lane == 0) s_wball[warp][a.R + g] = ball;
       });
   }
   __syncthreads();
@@ -364,7 +393,59 @@ __global__ void __launch_bounds__(kTile) layout_place_kernel(LayoutArgs a, Devic
   const bool live = t < a.T;
   const unsigned lt = lanemask_lt();
   const size_t tk = (size_t)t * a.k;
-  if (a.mode == MOE_LAYOUT_PER_PICK || a.mode == MOE_LAYOUT_DEDUP) {
+  if (a.mode != MOE_LAYOUT_PER_PICK) {
+    // mask bins: each lane walks its own ranks (and groups) in ascending order;
+    // its position in a bin is the count of earlier lanes in the bin's ballot
+    auto row_of = [&](int bin) {
+      return s_base[bin] + s_wcnt[warp][bin] + __popc(s_wball[warp][bin] & lt);
+    };
+    if (a.mode == MOE_LAYOUT_TWO_HOP) {
+      int cg = 0;
+      for (unsigned long long m = p.gmask; m; m &= m - 1, ++cg) {
+        const int g = __ffsll((long long)m) - 1;
+        const int row1 = row_of(a.R + g);
+        if (row1 < L.capacity_hop1) {
+          L.hop1_row_token[row1] = t;
+          L.token_groups[tk + cg] = row1;
+          const int nchild = __popcll(p.dmask & group_bits(g, a.rpg));
+          for (int ci = nchild; ci < a.k; ++ci) L.hop1_children[(size_t)row1 * a.k + ci] = -1;
+        } else {
+          L.token_groups[tk + cg] = -1;
+          over = true;
+        }
+      }
+      if (live)
+        for (int c = cg; c < a.k; ++c) L.token_groups[tk + c] = -1;
+    }
+    int c = 0;
+    for (unsigned long long m = p.dmask; m; m &= m - 1, ++c) {
+      const int r = __ffsll((long long)m) - 1;
+      const int row = row_of(r);
+      float coef = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if ((p.present >> j & 1u) && p.r[j] == r) coef += p.w[j];
+      const bool fits = row < L.capacity;
+      if (fits) {
+        L.row_token[row] = t;
+        L.row_coef[row] = coef;
+        L.token_rows[tk + c] = row;
+      } else {
+        L.token_rows[tk + c] = -1;
+        over = true;
+      }
+      if (a.mode == MOE_LAYOUT_TWO_HOP) {
+        const int g = r / a.rpg;
+        int row1 = row_of(a.R + g);
+        if (row1 >= L.capacity_hop1) row1 = -1;
+        const int ci = __popcll(p.dmask & group_bits(g, a.rpg) & ((1ull << r) - 1ull));
+        if (fits) L.hop2_src_row[row] = row1;
+        if (row1 >= 0) L.hop1_children[(size_t)row1 * a.k + ci] = fits ? row : -1;
+      }
+    }
+    if (live)
+      for (int cc = c; cc < a.k; ++cc) L.token_rows[tk + cc] = -1;
+  } else if (a.mode == MOE_LAYOUT_PER_PICK) {
     int cnt = 0;
     auto write_row = [&](int bin, bool has, unsigned ball, int c, uint32_t matched) {
       if (!has) return;
@@ -383,66 +464,11 @@ __global__ void __launch_bounds__(kTile) layout_place_kernel(LayoutArgs a, Devic
       }
       cnt = c + 1;
     };
-    if (a.mode == MOE_LAYOUT_PER_PICK)
-      warp_merge<KM, kPassPick>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int c, uint32_t m) {
-        write_row(key_bin<kPassPick>(b, a.R), has, ball, c, m);
-      });
-    else
-      warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int c, uint32_t m) {
-        write_row(key_bin<kPassRank>(b, a.R), has, ball, c, m);
-      });
+    warp_merge<KM, kPassPick>(p, a.rpg, [&](uint32_t b, bool has, unsigned ball, int c, uint32_t m) {
+      write_row(key_bin<kPassPick>(b, a.R), has, ball, c, m);
+    });
     if (live)
       for (int c = cnt; c < a.k; ++c) L.token_rows[tk + c] = -1;
-  } else {
-    // TWO_HOP: hop-1 (group) rows first, then hop-2 (rank) rows
-    unsigned long long gmask = 0;
-    int ng = 0;
-    warp_merge<KM, kPassGroup>(p, a.rpg, [&](uint32_t g, bool has, unsigned ball, int c, uint32_t) {
-      if (!has) return;
-      const int bin = key_bin<kPassGroup>(g, a.R);
-      const int row1 = s_base[bin] + s_wcnt[warp][bin] + __popc(ball & lt);
-      gmask |= 1ull << g;
-      ng = c + 1;
-      if (row1 < L.capacity_hop1) {
-        L.hop1_row_token[row1] = t;
-        L.token_groups[tk + c] = row1;
-        const int nchild = __popcll(p.dmask & group_bits((int)g, a.rpg));
-        for (int ci = nchild; ci < a.k; ++ci) L.hop1_children[(size_t)row1 * a.k + ci] = -1;
-      } else {
-        L.token_groups[tk + c] = -1;
-        over = true;
-      }
-    });
-    if (live)
-      for (int c = ng; c < a.k; ++c) L.token_groups[tk + c] = -1;
-    int nr = 0;
-    warp_merge<KM, kPassRank>(p, a.rpg, [&](uint32_t r, bool has, unsigned ball, int c, uint32_t matched) {
-      if (!has) return;
-      const int bin = key_bin<kPassRank>(r, a.R);
-      const int row = s_base[bin] + s_wcnt[warp][bin] + __popc(ball & lt);
-      float coef = 0.0f;
-#pragma unroll
-      for (int j = 0; j < KM; ++j)
-        if (matched >> j & 1u) coef += p.w[j];
-      const int g = (int)r / a.rpg;
-      const int gi = __popcll(gmask & ((1ull << g) - 1ull));
-      const int row1 = L.token_groups[tk + gi];
-      const int ci = __popcll(p.dmask & group_bits(g, a.rpg) & ((1ull << r) - 1ull));
-      nr = c + 1;
-      if (row < L.capacity) {
-        L.row_token[row] = t;
-        L.row_coef[row] = coef;
-        L.token_rows[tk + c] = row;
-        L.hop2_src_row[row] = row1;
-        if (row1 >= 0) L.hop1_children[(size_t)row1 * a.k + ci] = row;
-      } else {
-        L.token_rows[tk + c] = -1;
-        if (row1 >= 0) L.hop1_children[(size_t)row1 * a.k + ci] = -1;
-        over = true;
-      }
-    });
-    if (live)
-      for (int c = nr; c < a.k; ++c) L.token_rows[tk + c] = -1;
   }
   if (over) set_status(ctx.status, MOE_ERR_CAPACITY);
 }

@@ -10,10 +10,8 @@
 // column vectors with all of the item's rows in flight at once
 // (ld.global.nc.L1::no_allocate), multiply-adds them in row order and writes
 // the result once.  No atomics: the result does not depend on scheduling.
-//   one-hop:        items = tokens, lists = token_rows
-//   TWO_HOP hop 2:  items = hop-1 rows, lists = hop1_children, output = the
-//                   hop-1 buffer in the activation dtype (the group partial)
-//   TWO_HOP hop 1:  items = tokens, lists = token_groups, coefficients 1
+// Items are tokens and lists token_rows.  The two-hop reverse has its own
+// kernel below (both hops in one pass per token).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -142,6 +140,134 @@ __global__ void __launch_bounds__(256) fanin_kernel(FaninArgs a, DeviceCtx ctx) 
   if (bounds) set_status(ctx.status, MOE_ERR_BOUNDS);
 }
 
+// Rounds a float32 value to the activation dtype and back (the wire format).
+template <typename T>
+__device__ __forceinline__ float round_wire(float x);
+template <>
+__device__ __forceinline__ float round_wire<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float round_wire<__nv_bfloat16>(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+template <>
+__device__ __forceinline__ float round_wire<__half>(float x) {
+  return __half2float(__float2half_rn(x));
+}
+
+struct TwoHopArgs {
+  const uint8_t *y;         // hop-2 (rank) rows
+  uint32_t rb_in;
+  uint8_t *out;             // [T][H] of the output dtype
+  uint32_t rb_out;
+  uint8_t *hop1;            // group partials [rows1][H] in the input dtype, or null
+  int T, k;
+  const int *token_rows;    // [T][k] hop-2 rows of each token, ascending (grouped by group)
+  const int *hop2_src_row;  // hop-1 row of each hop-2 row
+  const float *coef;
+  int cap, cap1;
+  int nvec;
+};
+
+// TWO_HOP reverse in one pass per token, one warp per token: the token's rank
+// rows are summed group by group in float32 (ascending rows), each group
+// partial is rounded to the activation dtype (the slow-fabric wire format),
+// stored to its hop-1 row when a buffer is given, and the rounded partials are
+// summed in ascending group order into the token.  Bit-identical to running
+// the two reverse hops one after the other, without re-reading the partials.
+template <typename Tin, typename Tout, int KM>
+__global__ void __launch_bounds__(256) two_hop_fanin_kernel(TwoHopArgs a, DeviceCtx ctx) {
+  constexpr int VE = Elem<Tin>::kPerVec;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  bool bounds = false;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < a.T; t += gridDim.x * wpb) {
+    int my_r = -1, my_s = -1;
+    float my_c = 0.0f;
+    if (lane < a.k) {
+      my_r = __ldcs(a.token_rows + (size_t)t * a.k + lane);
+      if (my_r >= a.cap || my_r < -1) {
+        bounds = true;
+        my_r = -1;
+      }
+      if (my_r >= 0) {
+        my_c = __ldg(a.coef + my_r);
+        my_s = __ldg(a.hop2_src_row + my_r);
+        if (my_s >= a.cap1 || my_s < -1) {
+          bounds = true;
+          my_s = -1;
+        }
+      }
+    }
+    const unsigned vmask = __ballot_sync(kFull, my_r >= 0);
+    const int next_s = __shfl_down_sync(kFull, my_s, 1);
+    // a row closes its group when the next row belongs to another hop-1 row
+    const bool closes = my_r >= 0 && (!(vmask >> (lane + 1) & 1u) || lane == 31 || next_s != my_s);
+    const unsigned lastmask = __ballot_sync(kFull, closes);
+    int rows[KM], src[KM];
+    float cf[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      rows[j] = __shfl_sync(kFull, my_r, j);
+      src[j] = __shfl_sync(kFull, my_s, j);
+      cf[j] = __shfl_sync(kFull, my_c, j);
+    }
+    uint8_t *orow = a.out + (size_t)t * a.rb_out;
+    for (int v = lane; v < a.nvec; v += 32) {
+      uint4 d[KM];
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (vmask >> j & 1u) d[j] = ld_stream_v4(a.y + (size_t)rows[j] * a.rb_in + (size_t)v * 16);
+      float acc_g[VE], acc_o[VE];
+#pragma unroll
+      for (int e = 0; e < VE; ++e) acc_g[e] = acc_o[e] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        if (vmask >> j & 1u)
+#pragma unroll
+          for (int e = 0; e < VE; ++e) acc_g[e] = fmaf(cf[j], Elem<Tin>::get(d[j], e), acc_g[e]);
+        if (lastmask >> j & 1u) {
+#pragma unroll
+          for (int e = 0; e < VE; ++e) acc_g[e] = round_wire<Tin>(acc_g[e]);
+          if (a.hop1 && src[j] >= 0)
+            store_out<Tin, VE>(a.hop1 + (size_t)src[j] * a.rb_in + (size_t)v * 16, acc_g);
+#pragma unroll
+          for (int e = 0; e < VE; ++e) {
+            acc_o[e] += acc_g[e];
+            acc_g[e] = 0.0f;
+          }
+        }
+      }
+      store_out<Tout, VE>(orow + (size_t)v * VE * sizeof(Tout), acc_o);
+    }
+  }
+  if (bounds) set_status(ctx.status, MOE_ERR_BOUNDS);
+}
+
+template <typename Tin, typename Tout, int KM>
+cudaError_t launch_two_hop3(const TwoHopArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+  const int wpb = 8;
+  long blocks = ((long)a.T + wpb - 1) / wpb;
+  const long cap = (long)ctx.num_sms * 16;
+  if (blocks > cap) blocks = cap;
+  two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, wpb * 32, 0, s>>>(a, ctx);
+  return count_launch(cudaGetLastError());
+}
+
+template <typename Tin, typename Tout>
+cudaError_t launch_two_hop2(const TwoHopArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+  if (a.k <= 2) return launch_two_hop3<Tin, Tout, 2>(a, ctx, s);
+  if (a.k <= 4) return launch_two_hop3<Tin, Tout, 4>(a, ctx, s);
+  if (a.k <= 8) return launch_two_hop3<Tin, Tout, 8>(a, ctx, s);
+  return launch_two_hop3<Tin, Tout, 16>(a, ctx, s);
+}
+
+template <typename Tin>
+cudaError_t launch_two_hop1(const TwoHopArgs &a, int out_dtype, const DeviceCtx &ctx, cudaStream_t s) {
+  if (out_dtype == MOE_F16) return launch_two_hop2<Tin, __half>(a, ctx, s);
+  if (out_dtype == MOE_BF16) return launch_two_hop2<Tin, __nv_bfloat16>(a, ctx, s);
+  return launch_two_hop2<Tin, float>(a, ctx, s);
+}
+
 template <typename Tin, typename Tout, int KM>
 cudaError_t launch3(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   const int wpb = 8;
@@ -200,30 +326,25 @@ cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
     a.nvec = (int)(a.rb_in / 16);
     return launch_fanin(a, dtype, out_dtype, ctx, s);
   }
-  // hop 2 reverse: rank rows -> group partials in the activation dtype
-  a.y = static_cast<const uint8_t *>(y);
-  a.rb_in = (uint32_t)((size_t)H * elem_size(dtype));
-  a.out = static_cast<uint8_t *>(hop1_buf);
-  a.rb_out = a.rb_in;
-  a.n_items = -1;
-  a.n_items_dev = L.num_rows_hop1;
-  a.cap_items = L.capacity_hop1;
-  a.lists = L.hop1_children;
-  a.coef = coef;
-  a.src_cap = L.capacity;
-  a.nvec = (int)(a.rb_in / 16);
-  cudaError_t err = launch_fanin(a, dtype, dtype, ctx, s);
-  if (err != cudaSuccess) return err;
-  // hop 1 reverse: group partials -> token
-  a.y = static_cast<const uint8_t *>(hop1_buf);
-  a.out = static_cast<uint8_t *>(out);
-  a.rb_out = (uint32_t)((size_t)H * elem_size(out_dtype));
-  a.n_items = L.T;
-  a.n_items_dev = nullptr;
-  a.lists = L.token_groups;
-  a.coef = nullptr;
-  a.src_cap = L.capacity_hop1;
-  return launch_fanin(a, dtype, out_dtype, ctx, s);
+  // both reverse hops in one pass per token
+  TwoHopArgs b;
+  b.y = static_cast<const uint8_t *>(y);
+  b.rb_in = (uint32_t)((size_t)H * elem_size(dtype));
+  b.out = static_cast<uint8_t *>(out);
+  b.rb_out = (uint32_t)((size_t)H * elem_size(out_dtype));
+  b.hop1 = static_cast<uint8_t *>(hop1_buf);
+  b.T = L.T;
+  b.k = L.k;
+  b.token_rows = L.token_rows;
+  b.hop2_src_row = L.hop2_src_row;
+  b.coef = coef;
+  b.cap = L.capacity;
+  b.cap1 = L.capacity_hop1;
+  b.nvec = (int)(b.rb_in / 16);
+  if (b.T == 0) return cudaSuccess;
+  if (dtype == MOE_F16) return launch_two_hop1<__half>(b, out_dtype, ctx, s);
+  if (dtype == MOE_BF16) return launch_two_hop1<__nv_bfloat16>(b, out_dtype, ctx, s);
+  return launch_two_hop1<float>(b, out_dtype, ctx, s);
 }
 
 }  // namespace moe

@@ -209,10 +209,7 @@ static int check_layout_shape(const moe_layout *L) {
   if (L->T < 0 || !valid_ekr(L->E, L->k) || L->R < 1 || L->R > moe::kMaxR) return MOE_ERR_INVALID_ARG;
   if (L->mode < MOE_LAYOUT_PER_PICK || L->mode > MOE_LAYOUT_TWO_HOP) return MOE_ERR_INVALID_ARG;
   if (L->T > 0 && !L->token_rows) return MOE_ERR_INVALID_ARG;
-  if (L->mode == MOE_LAYOUT_TWO_HOP &&
-      (!L->num_rows_hop1 || (L->T > 0 && !L->token_groups) ||
-       (L->capacity_hop1 > 0 && !L->hop1_children)))
-    return MOE_ERR_INVALID_ARG;
+  if (L->mode == MOE_LAYOUT_TWO_HOP && (L->T > 0 && !L->token_groups)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -246,9 +243,10 @@ int moe_combine(const void *y, int32_t dtype, int32_t H, const moe_layout *layou
   if (layout->T > 0 && (!out || !aligned16(out))) return MOE_ERR_INVALID_ARG;
   if (layout->capacity > 0 && (!y || !aligned16(y))) return MOE_ERR_INVALID_ARG;
   if (!row_coef && layout->capacity > 0 && !layout->row_coef) return MOE_ERR_INVALID_ARG;
-  if (layout->mode == MOE_LAYOUT_TWO_HOP && layout->capacity_hop1 > 0 &&
-      (!hop1_buf || !aligned16(hop1_buf)))
-    return MOE_ERR_INVALID_ARG;
+  if (layout->mode == MOE_LAYOUT_TWO_HOP) {
+    if (hop1_buf && !aligned16(hop1_buf)) return MOE_ERR_INVALID_ARG;
+    if (layout->capacity > 0 && !layout->hop2_src_row) return MOE_ERR_INVALID_ARG;
+  }
   moe::DeviceCtx ctx;
   rc = get_ctx(&ctx);
   if (rc) return rc;

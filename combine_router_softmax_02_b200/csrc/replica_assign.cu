@@ -8,14 +8,20 @@
 // lower slot id.
 //
 // The whole CTA stages the demand vector and the replica map in shared memory
-// (each replica entry pre-packed as rank << 15 | slot); warp 0 then runs the
-// serial greedy.  For each active expert the lanes form the key
+// (each replica entry pre-packed as rank << 15 | slot).  Warp 0 then walks the
+// experts 32 at a time.  An expert with one valid replica has no choice: its
+// rank only gains one activated expert, so the forced experts between two
+// experts with a choice are applied together with shared-memory atomics.  For
+// an expert with a choice the lanes form the key
 // activated[rank] << 21 | rank << 15 | slot of its replicas and one
 // redux.sync.min picks the winner, so the tie rules are the key's bit order.
+// The serial chain is only as long as the number of experts with a choice.
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
 
 __global__ void __launch_bounds__(256) replica_assign_kernel(
     const int *__restrict__ counts, int E, const int *__restrict__ off,
@@ -45,37 +51,64 @@ __global__ void __launch_bounds__(256) replica_assign_kernel(
 
   const int lane = threadIdx.x;
   bool bad = false;
-  for (int e = 0; e < E; ++e) {
-    const int c = s_cnt[e];
-    int lo = s_off[e], hi = s_off[e + 1];
-    if (c < 0) bad = true;
-    if (lo < 0 || hi > n_entries || lo > hi) {
-      bad = true;
-      lo = hi = 0;
+  for (int base = 0; base < E; base += 32) {
+    // classify this lane's expert: inactive, forced (one valid replica), or a choice
+    const int e = base + lane;
+    int kind = 0;        // 0 inactive / out of range, 1 forced, 2 choice
+    int fkey = -1;       // the forced expert's key
+    int lo = 0, hi = 0;
+    if (e < E) {
+      const int c = s_cnt[e];
+      lo = s_off[e];
+      hi = s_off[e + 1];
+      if (c < 0 || lo < 0 || hi > n_entries || lo > hi) {
+        bad = true;
+        lo = hi = 0;
+      }
+      if (c > 0) {
+        int nvalid = 0;
+        for (int i = lo; i < hi && nvalid < 2; ++i)
+          if (s_key[i] >= 0) {
+            ++nvalid;
+            fkey = s_key[i];
+          }
+        if (nvalid == 0) bad = true;  // active expert without a valid replica
+        kind = (nvalid == 0) ? 0 : (nvalid == 1 ? 1 : 2);
+      }
     }
-    unsigned best = 0xffffffffu;
-    if (c > 0) {
-      for (int i = lo + lane; i < hi; i += 32) {
+    unsigned choice = __ballot_sync(kFull, kind == 2);
+    int done_below = 0;  // forced lanes below this index are already applied
+    while (true) {
+      const int m = choice ? __ffs(choice) - 1 : 32;
+      if (kind == 1 && lane >= done_below && lane < m) atomicAdd(&s_active[fkey >> 15], 1);
+      __syncwarp();
+      if (m == 32) break;
+      // expert base + m has a choice: evaluate its replicas against the counts so far
+      const int me = base + m;
+      const int mlo = __shfl_sync(kFull, lo, m), mhi = __shfl_sync(kFull, hi, m);
+      unsigned best = 0xffffffffu;
+      for (int i = mlo + lane; i < mhi; i += 32) {
         const int kb = s_key[i];
         if (kb >= 0) best = min(best, ((unsigned)s_active[kb >> 15] << 21) | (unsigned)kb);
       }
-      best = __reduce_min_sync(0xffffffffu, best);
-    }
-    if (lane == 0) {
-      if (c > 0 && best != 0xffffffffu) {
+      best = __reduce_min_sync(kFull, best);
+      if (lane == 0) {
         const int r = (best >> 15) & 63;
-        expert_slot[e] = best & 0x7fff;
-        expert_rank[e] = r;
+        expert_slot[me] = best & 0x7fff;
+        expert_rank[me] = r;
         s_active[r] += 1;
-      } else {
-        if (c > 0) bad = true;  // active expert without a valid replica
-        expert_slot[e] = -1;
-        expert_rank[e] = -1;
       }
+      __syncwarp();
+      done_below = m + 1;
+      choice &= choice - 1;
     }
-    __syncwarp();
+    if (e < E && kind != 2) {
+      expert_slot[e] = (kind == 1) ? (fkey & 0x7fff) : -1;
+      expert_rank[e] = (kind == 1) ? (fkey >> 15) : -1;
+    }
   }
-  if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
+  if (__any_sync(kFull, bad) && lane == 0) set_status(ctx.status, MOE_ERR_BAD_INPUT);
+  __syncwarp();
   for (int r = lane; r < R; r += 32) rank_active[r] = s_active[r];
 }
 

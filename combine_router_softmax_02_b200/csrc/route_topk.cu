@@ -7,10 +7,14 @@
 //
 // Lane l holds experts l, l+32, l+64, ... of its token (coalesced 128-byte
 // loads).  Softmax max and sum are butterfly reductions, so every lane ends
-// with bit-identical values.  Each top-k round takes the lane's best
-// remaining expert, then two redux.sync instructions find the warp winner:
-// the largest order-preserving key of the logit, and among equal keys the
-// smallest expert id (ties to the lower index).
+// with bit-identical values.  Selection works on an order-preserving u32 key
+// of each logit.  The k-th largest of the 32 lane maxima is a lower bound on
+// the k-th largest key, so only the few elements at or above it can be picked;
+// they are compacted one per lane through shared memory and k rounds of two
+// redux.sync instructions pick the winners: the largest key, and among equal
+// keys the smallest expert id (ties to the lower index).  When more than 32
+// elements tie at the bound, every element is scanned each round instead.
+// The gate weights are computed at the end, one pick per lane.
 #include <math.h>
 
 #include "moe_internal.cuh"
@@ -26,6 +30,11 @@ constexpr unsigned kFull = 0xffffffffu;
 __device__ __forceinline__ uint32_t order_key(float v) {
   uint32_t u = (v == 0.0f) ? 0u : __float_as_uint(v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inverse of order_key (a zero key comes back as +0).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -45,7 +54,10 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          int E, int k, int n_groups, int gpt,
                                                          int renorm, int *__restrict__ idx_out,
                                                          float *__restrict__ w_out, DeviceCtx ctx) {
+  __shared__ uint32_t s_ck[8][32];  // per-warp candidate keys
+  __shared__ int s_ce[8][32];       // and their experts
   const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int wpb = blockDim.x >> 5;
   const bool limit = gpt > 0 && gpt < n_groups;
   const int gsize = limit ? E / n_groups : E;
@@ -107,30 +119,84 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
         if (!(keep >> gid[j] & 1u)) avail &= ~(1u << j);
     }
 
-    int my_e = 0;
-    float my_w = 0.0f;
-    for (int r = 0; r < k; ++r) {
-      uint32_t bk = 0;
-      int be = 0x7fffffff;
-      float bv = 0.0f;
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        if ((avail >> j & 1u) && key[j] > bk) {  // strict: lowest slot wins ties
-          bk = key[j];
-          be = lane + 32 * j;
-          bv = v[j];
+    for (int j = 0; j < EPL; ++j)
+      if (!(avail >> j & 1u)) key[j] = 0;  // 0 = not a candidate
+
+    // Candidates.  tau = the k-th largest of the 32 lane maxima: k distinct
+    // elements reach it, so every top-k element has key >= tau.
+    uint32_t lm = 0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) lm = max(lm, key[j]);
+    uint32_t tau = 0;
+    for (int r = 0; r < k; ++r) {
+      tau = __reduce_max_sync(kFull, lm);
+      const unsigned lw = __reduce_min_sync(kFull, lm == tau ? (unsigned)lane : 32u);
+      if (lane == (int)lw) lm = 0;
+    }
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) cnt += (key[j] >= tau) ? 1 : 0;
+    const unsigned total = __reduce_add_sync(kFull, (unsigned)cnt);
+
+    int my_e = 0;
+    uint32_t my_k = 0;
+    if (total <= 32) {
+      // one candidate per lane, through shared memory, then k rounds of
+      // (largest key, then smallest expert id among equal keys)
+      int pos = cnt;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int n = __shfl_up_sync(kFull, pos, d);
+        if (lane >= d) pos += n;
+      }
+      pos -= cnt;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (key[j] >= tau) {
+          s_ck[warp][pos] = key[j];
+          s_ce[warp][pos] = lane + 32 * j;
+          ++pos;
+        }
+      __syncwarp();
+      uint32_t ck = lane < (int)total ? s_ck[warp][lane] : 0u;
+      const unsigned ce = lane < (int)total ? (unsigned)s_ce[warp][lane] : 0x7fffffffu;
+      __syncwarp();
+      for (int r = 0; r < k; ++r) {
+        const uint32_t kmax = __reduce_max_sync(kFull, ck);
+        const unsigned ewin = __reduce_min_sync(kFull, ck == kmax ? ce : 0x7fffffffu);
+        if (ce == ewin) ck = 0;
+        if (lane == r) {
+          my_e = (int)ewin;
+          my_k = kmax;
         }
       }
-      const uint32_t kmax = __reduce_max_sync(kFull, bk);
-      const int ewin = (int)__reduce_min_sync(kFull, (bk == kmax) ? (unsigned)be : 0x7fffffffu);
-      const int owner = ewin & 31;
-      const float vwin = __shfl_sync(kFull, bv, owner);
-      if (lane == owner) avail &= ~(1u << (ewin >> 5));
-      if (lane == r) {
-        my_e = ewin;
-        my_w = expf(vwin - m) / s;
+    } else {
+      // many ties at tau: scan every element each round
+      for (int r = 0; r < k; ++r) {
+        uint32_t bk = 0;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j)
+          if (key[j] > bk) {  // strict: the lowest slot wins ties
+            bk = key[j];
+            be = lane + 32 * j;
+          }
+        const uint32_t kmax = __reduce_max_sync(kFull, bk);
+        const int ewin = (int)__reduce_min_sync(kFull, (bk == kmax) ? (unsigned)be : 0x7fffffffu);
+        if (lane == (ewin & 31)) {
+#pragma unroll
+          for (int j = 0; j < EPL; ++j)
+            if (j == (ewin >> 5)) key[j] = 0;
+        }
+        if (lane == r) {
+          my_e = ewin;
+          my_k = kmax;
+        }
       }
     }
+    // gate weights, one per lane: softmax probability of the pick
+    float my_w = (lane < k) ? expf(key_value(my_k) - m) / s : 0.0f;
     if (renorm) {
       const float tot = warp_sum(lane < k ? my_w : 0.0f);
       my_w = my_w / tot;

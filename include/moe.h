@@ -221,7 +221,8 @@ MOE_API int moe_build_layout_static(const int32_t *topk_idx, const float *topk_w
  * AllToAll for MoE decode", section "Work the 8-GPU payload example").
  * x [T][H] of `dtype`; packed [capacity][H].  TWO_HOP: packed_hop1
  * [capacity_hop1][H] receives the hop-1 (group) rows and packed the hop-2
- * (rank) rows, forwarded from packed_hop1; packed_hop1 is ignored otherwise.
+ * (rank) rows, which equal the group rows they are forwarded from; both are
+ * written from one read of each token.  packed_hop1 is ignored otherwise.
  */
 MOE_API int moe_pack(const void *x, int32_t dtype, int32_t H, const moe_layout *layout,
              void *packed, void *packed_hop1, moe_stream_t stream);
@@ -233,10 +234,12 @@ MOE_API int moe_pack(const void *x, int32_t dtype, int32_t H, const moe_layout *
  * decode", section "changes the routing information").
  * y [capacity][H] of `dtype` (expert outputs, one per row); row_coef [capacity]
  * or NULL for layout->row_coef; out [T][H] of out_dtype.
- * TWO_HOP: the reverse of the two hops.  hop1_buf [capacity_hop1][H] of `dtype`
- * receives each group partial sum over the group's rank rows (rounded to
- * `dtype`, the dtype that would cross the slow fabric), then out[t] = sum of
- * t's group partials.  hop1_buf is ignored for the other modes.
+ * TWO_HOP: the reverse of the two hops, in one pass per token.  Each group
+ * partial, the sum over the group's rank rows in ascending order, is rounded to
+ * `dtype` (the dtype that would cross the slow fabric); out[t] = the sum of t's
+ * rounded group partials in ascending group order.  hop1_buf [capacity_hop1][H]
+ * of `dtype` receives the group partials at their hop-1 rows, or is NULL to
+ * skip storing them.  hop1_buf is ignored for the other modes.
  */
 MOE_API int moe_combine(const void *y, int32_t dtype, int32_t H, const moe_layout *layout,
                 const float *row_coef, void *out, int32_t out_dtype, void *hop1_buf,

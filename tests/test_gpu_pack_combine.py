@@ -158,6 +158,17 @@ def check_two_hop(moe, cfg, sample=None):
             extra[have] += oracle.ulp(z, fmt)
     assert_close_combine(out[torch.from_numpy(toks).cuda()].double().cpu().numpy(), o, absum, fmt,
                          extra=extra, what="two-hop combine")
+    # the stored group partials: each within its own bound of the oracle's rounded partial
+    z_dev = dc.hop1_buf[torch.from_numpy(used1.astype(np.int64)).cuda()].double().cpu().numpy()
+    z_ref = np.stack([zs[i] for i in range(len(used1))])
+    zabs = np.zeros_like(z_ref)
+    for i2, s1 in enumerate(sub["hop2_src_row"]):
+        zabs[s1] += np.abs(c2[i2] * y2[i2])
+    assert_close_combine(z_dev, z_ref, zabs, fmt, extra=oracle.ulp(z_ref, fmt), what="group partials")
+    # not storing the partials changes nothing else
+    out2 = moe.combine(dc.packed, dc.layout, out_dtype=dc.out_dtype, store_hop1=False)
+    assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
+    assert moe.get_status() == 0
 
 
 def test_two_hop_small_every_row(moe):
