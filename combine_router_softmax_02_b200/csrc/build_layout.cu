@@ -171,8 +171,12 @@ __device__ __forceinline__ unsigned long long group_bits(int g, int rpg) {
 }
 
 // ------------------------------------------------------------- finalize ----
-// Runs in the last count block: segment offsets and the host-visible offsets.
-__device__ void finalize(const LayoutArgs &a, const int *s_er, DeviceCtx ctx) {
+// Runs in the last count block, all threads: the totals are loaded into
+// shared memory in parallel (tot), then thread 0 scans them into segment
+// offsets and the host-visible offsets.
+__device__ void finalize(const LayoutArgs &a, const int *s_er, int *tot, DeviceCtx ctx) {
+  for (int i = threadIdx.x; i < a.NB; i += blockDim.x) tot[i] = __ldcg(a.totals + i);
+  __syncthreads();
   if (threadIdx.x != 0) return;
   const moe_layout &L = a.L;
   if (a.mode == MOE_LAYOUT_PER_PICK) {
@@ -180,20 +184,20 @@ __device__ void finalize(const LayoutArgs &a, const int *s_er, DeviceCtx ctx) {
     for (int r = 0; r <= a.R; ++r) base[r] = 0;
     for (int e = 0; e < a.E; ++e) {
       const int r = s_er[e];
-      if ((unsigned)r < (unsigned)a.R) base[r + 1] += __ldcg(a.totals + e);
+      if ((unsigned)r < (unsigned)a.R) base[r + 1] += tot[e];
     }
     for (int r = 0; r < a.R; ++r) base[r + 1] += base[r];
     for (int r = 0; r <= a.R; ++r) L.rank_offsets[r] = base[r];
+    const int n = base[a.R];
     for (int e = 0; e < a.E; ++e) {
       const int r = s_er[e];
       if ((unsigned)r < (unsigned)a.R) {
         a.seg_off[e] = base[r];
-        base[r] += __ldcg(a.totals + e);
+        base[r] += tot[e];
       } else {
         a.seg_off[e] = 0;
       }
     }
-    const int n = L.rank_offsets[a.R];
     *L.num_rows = n;
     if (n > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
     return;
@@ -202,7 +206,7 @@ __device__ void finalize(const LayoutArgs &a, const int *s_er, DeviceCtx ctx) {
   for (int r = 0; r < a.R; ++r) {
     a.seg_off[r] = run;
     L.rank_offsets[r] = run;
-    run += __ldcg(a.totals + r);
+    run += tot[r];
   }
   L.rank_offsets[a.R] = run;
   *L.num_rows = run;
@@ -212,7 +216,7 @@ __device__ void finalize(const LayoutArgs &a, const int *s_er, DeviceCtx ctx) {
     for (int g = 0; g < a.G; ++g) {
       a.seg_off[a.R + g] = run1;
       L.group_offsets[g] = run1;
-      run1 += __ldcg(a.totals + a.R + g);
+      run1 += tot[a.R + g];
     }
     L.group_offsets[a.G] = run1;
     *L.num_rows_hop1 = run1;
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(kTile) layout_count_kernel(LayoutArgs a, Devic
   __syncthreads();
   if (s_last) {
     __threadfence();
-    finalize(a, s_er, ctx);
+    finalize(a, s_er, s_cnt, ctx);  // s_cnt is free again after the flush
   }
 }
 

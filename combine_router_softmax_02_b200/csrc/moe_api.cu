@@ -6,7 +6,6 @@
 #include "moe_internal.cuh"
 
 namespace moe {
-size_t fanout_max_row_bytes();
 std::atomic<unsigned long long> g_kernel_launches{0};
 }
 
@@ -220,7 +219,7 @@ int moe_pack(const void *x, int32_t dtype, int32_t H, const moe_layout *layout, 
   if (!valid_dtype(dtype) || H < 1) return MOE_ERR_INVALID_ARG;
   const size_t rb = (size_t)H * elem_bytes(dtype);
   if (rb % 16 != 0) return MOE_ERR_UNSUPPORTED;
-  if (rb > moe::fanout_max_row_bytes()) return MOE_ERR_UNSUPPORTED;
+  if (rb > ((size_t)1 << 30)) return MOE_ERR_UNSUPPORTED;
   if (layout->T > 0 && (!x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
   if (layout->capacity > 0 && (!packed || !aligned16(packed))) return MOE_ERR_INVALID_ARG;
   if (layout->mode == MOE_LAYOUT_TWO_HOP && layout->capacity_hop1 > 0 &&
