@@ -194,18 +194,66 @@ def optimal_max_active(counts, replica_offsets, replica_slots, slot_rank, R: int
     return 0 if best is None else best
 
 
-def token_balanced_active(counts, replica_offsets, replica_slots, slot_rank, R: int) -> np.ndarray:
-    """Activated replicas per rank when every expert's tokens are split as
-    evenly as possible over all its replicas (the token-balancing policy the
-    page compares METRO with): a replica is activated when it gets >= 1 token.
-    Tokens of expert e go round-robin over its slots in ascending slot order."""
+def token_balanced_split(counts, replica_offsets, replica_slots, slot_rank, R: int, S: int):
+    """Token-balanced routing, the comparison policy of "METRO AllGather vs
+    AllToAll for MoE decode" (sections "Add the expert-weight traffic term" and
+    "Know what the paper actually measured": EPLB token routing, which spreads
+    an expert's tokens over its replicas).  The c tokens of expert e are dealt
+    round-robin over its n replicas in ascending slot id, so the i-th replica
+    gets floor(c / n) + (1 if i < c mod n else 0) tokens; a replica with at
+    least one token is activated.
+
+    Returns ``slot_tokens`` (int64 [S]) and ``rank_active`` (int64 [R])."""
+    slot_tokens = np.zeros(S, np.int64)
     act = np.zeros(R, np.int64)
     for e in range(len(counts)):
-        slots = [int(s) for s in replica_slots[replica_offsets[e]:replica_offsets[e + 1]]]
-        for j, s in enumerate(slots):
-            if j < counts[e]:
+        c = int(counts[e])
+        slots = sorted(int(s) for s in replica_slots[replica_offsets[e]:replica_offsets[e + 1]])
+        if c <= 0 or not slots:
+            continue
+        n = len(slots)
+        for i, s in enumerate(slots):
+            slot_tokens[s] = c // n + (1 if i < c % n else 0)
+            if slot_tokens[s] > 0:
                 act[slot_rank[s]] += 1
-    return act
+    return slot_tokens, act
+
+
+def token_balanced_active(counts, replica_offsets, replica_slots, slot_rank, R: int) -> np.ndarray:
+    """Activated replicas per rank under token-balanced routing (above)."""
+    S = int(np.max(np.asarray(replica_slots), initial=-1)) + 1
+    return token_balanced_split(counts, replica_offsets, replica_slots, slot_rank, R, S)[1]
+
+
+# --------------------------------------------------------------------------
+# dispatch statistics of the send-count matrix
+# --------------------------------------------------------------------------
+def gini(x) -> float:
+    """Gini coefficient: sum over all ordered pairs |x_i - x_j| / (2 n^2 mean);
+    0 when every value is 0."""
+    x = np.asarray(x, np.float64)
+    n, tot = x.shape[0], x.sum()
+    if n == 0 or tot == 0:
+        return 0.0
+    return float(np.abs(x[:, None] - x[None, :]).sum() / (2.0 * n * n * (tot / n)))
+
+
+def dispatch_stats(counts, send_counts) -> Dict[str, float]:
+    """Scalar summaries of one dispatch (gist.science summary of DODOCO,
+    "Methodology": the per-expert max/mean ratio measures routing skew
+    independent of the expert-to-rank map; the Gini coefficient measures
+    per-rank load imbalance).  Per-rank load = rows each destination rank
+    receives (column sums of the send-count matrix S).  Also the share of rows
+    that stay on their source rank (the diagonal of S)."""
+    counts = np.asarray(counts, np.float64)
+    S = np.asarray(send_counts, np.float64)
+    load = S.sum(axis=0)
+    return {
+        "expert_max_mean": float(counts.max() / counts.mean()) if counts.sum() else 0.0,
+        "rank_gini": gini(load),
+        "rank_max_mean": float(load.max() / load.mean()) if load.sum() else 0.0,
+        "own_rank_row_share": float(np.trace(S) / S.sum()) if S.sum() else 0.0,
+    }
 
 
 # --------------------------------------------------------------------------

@@ -393,3 +393,60 @@ def check_round_to(round_to):
     assert np.array_equal(round_to(xf.astype(np.float64), "bf16"), ref)
     # ties to even
     assert round_to(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8]), "bf16").tolist() == [1.0, 1 + 2.0 ** -6]
+
+
+# ----------------------------------------------------------- statistics ----
+def check_gini(gini):
+    assert gini([3, 3, 3, 3]) == 0.0 and gini([0, 0]) == 0.0
+    for n in (2, 5, 64):                       # all load on one rank: (n - 1) / n
+        x = np.zeros(n)
+        x[n // 2] = 7
+        assert math.isclose(gini(x), (n - 1) / n, rel_tol=1e-14)
+    assert math.isclose(gini([1, 2, 3, 4]), 0.25, rel_tol=1e-14)   # 20 / (2 * 16 * 2.5)
+    # the closed form over sorted values: G = 2 sum_i i x_(i) / (n sum x) - (n + 1) / n
+    rng = np.random.default_rng(12)
+    for _ in range(20):
+        x = rng.integers(0, 50, size=int(rng.integers(2, 70))).astype(np.float64)
+        if x.sum() == 0:
+            continue
+        xs, n = np.sort(x), x.shape[0]
+        ref = 2 * np.sum(np.arange(1, n + 1) * xs) / (n * xs.sum()) - (n + 1) / n
+        assert math.isclose(gini(x), ref, rel_tol=1e-12, abs_tol=1e-15)
+        assert math.isclose(gini(3 * x), gini(x), rel_tol=1e-12, abs_tol=1e-15)   # scale free
+
+
+def check_dispatch_stats(dispatch_stats):
+    counts = np.array([1, 1, 1, 5])
+    S = np.array([[4, 1, 0], [0, 2, 2], [1, 0, 2]])     # loads 5, 3, 4
+    d = dispatch_stats(counts, S)
+    assert math.isclose(d["expert_max_mean"], 2.5)
+    assert math.isclose(d["rank_max_mean"], 5 / 4)
+    assert math.isclose(d["own_rank_row_share"], 8 / 12)
+    assert math.isclose(d["rank_gini"], (2 + 1 + 1) * 2 / (2 * 9 * 4))
+
+
+def check_token_balanced(token_balanced_split):
+    # conservation, near-equal split in ascending slot order, activation = min(c, n)
+    rng = np.random.default_rng(13)
+    for _ in range(30):
+        E, R = int(rng.integers(1, 20)), int(rng.integers(1, 9))
+        nrep = rng.integers(1, R + 1, size=E)
+        reps = [rng.choice(R, size=int(n), replace=False) for n in nrep]
+        sr = np.concatenate(reps).astype(np.int64)
+        S = sr.shape[0]
+        perm = rng.permutation(S)
+        sr_by = np.empty(S, np.int64)
+        sr_by[perm] = sr
+        off = np.zeros(E + 1, np.int64)
+        off[1:] = np.cumsum(nrep)
+        counts = rng.integers(0, 9, size=E)
+        st, act = token_balanced_split(counts, off, perm, sr_by, R, S)
+        exp_act = np.zeros(R, np.int64)
+        for e in range(E):
+            sl = sorted(perm[off[e]:off[e + 1]].tolist())
+            toks = [int(st[s]) for s in sl]
+            assert sum(toks) == counts[e]
+            assert max(toks) - min(toks) <= 1 and toks == sorted(toks, reverse=True)
+            for s in sl:
+                exp_act[sr_by[s]] += st[s] > 0
+        assert act.tolist() == exp_act.tolist()

@@ -145,3 +145,27 @@ def test_round_half_away_caught():
         return np.where(tie, np.sign(x) * (np.abs(r) + q * (np.abs(r) < np.abs(x))), r)
     with pytest.raises(AssertionError):
         pins.check_round_to(mutant)
+
+
+def test_gini_without_mean_normalisation_caught():
+    def mutant(x):
+        x = np.asarray(x, np.float64)
+        n = x.shape[0]
+        return float(np.abs(x[:, None] - x[None, :]).sum() / (2.0 * n * n)) if x.sum() else 0.0
+    with pytest.raises(AssertionError):
+        pins.check_gini(mutant)
+
+
+def test_token_balanced_listed_order_caught():
+    # deals tokens in the listed order instead of ascending slot id
+    def mutant(counts, off, slots, sr, R, S):
+        st = np.zeros(S, np.int64)
+        act = np.zeros(R, np.int64)
+        for e in range(len(counts)):
+            ls = [int(s) for s in slots[off[e]:off[e + 1]]]
+            for i, s in enumerate(ls):
+                st[s] = counts[e] // len(ls) + (1 if i < counts[e] % len(ls) else 0)
+                act[sr[s]] += st[s] > 0
+        return st, act
+    with pytest.raises(AssertionError):
+        pins.check_token_balanced(mutant)

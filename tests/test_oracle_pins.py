@@ -77,3 +77,26 @@ def test_pack_is_row_gather():
 def test_ulp():
     assert oracle.ulp(np.array([1.0, 1.5, 2.0]), "bf16").tolist() == [2.0 ** -7, 2.0 ** -7, 2.0 ** -6]
     assert oracle.ulp(np.array([1e-7]), "f16").tolist() == [2.0 ** -24]
+
+
+def test_gini_closed_forms():
+    pins.check_gini(oracle.gini)
+
+
+def test_dispatch_stats_hand_worked():
+    pins.check_dispatch_stats(oracle.dispatch_stats)
+
+
+def test_token_balanced_split():
+    pins.check_token_balanced(oracle.token_balanced_split)
+
+
+def test_uniform_own_row_share_single_pick():
+    """With top-1 routing on E/R experts per rank, the own-rank row share is the
+    own-rank pick share: 1/R in expectation (the 12.5% of one node of 8)."""
+    import workloads as W
+    cfg = W.CONFIGS["c1"].with_(T=8 * 4096, k=1)
+    idx, w = oracle.route_topk(W.make_logits(cfg, seed=5), 1)
+    L = oracle.build_layout(idx, w, W.expert_home_rank(cfg), cfg.T // 8, 8, oracle.DEDUP)
+    share = oracle.dispatch_stats(oracle.demand_hist(idx, cfg.E), L["send_counts"])["own_rank_row_share"]
+    assert abs(share - 0.125) < 5 * (0.125 * 0.875 / cfg.T) ** 0.5
