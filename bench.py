@@ -145,6 +145,8 @@ def step_bytes(cfg: W.Config, rows: int, rows_hop1: int, S: int) -> dict:
     else:
         d["pack"] = (T + rows) * H * b + T * k * 4
         d["combine"] = (rows + T) * H * b + rows * 4 + T * k * 4
+    # the fused front end reads the picks once less (no separate count pass)
+    d["route_layout"] = d["route_topk"] + d["build_layout"] - T * k * 4
     return d
 
 
@@ -175,29 +177,38 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     x = x_h.to(dev)
     stream = torch.cuda.current_stream(dev)
     names = ["route_topk", "demand_hist", "replica_assign", "build_layout", "pack", "combine"]
+    single = bool(np.all(np.diff(rm.replica_offsets) == 1))
+    if args.fused and not single:
+        raise SystemExit("--fused needs a placement with one replica per expert")
+    if args.fused:
+        names = ["route_layout", "pack", "combine"]
+        static_rank = torch.from_numpy(rm.slot_rank[rm.replica_slots]).to(dev, torch.int32)
 
     def one_step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        moe.route_topk(logits, cfg.k, cfg.n_groups, cfg.groups_per_token, False, dc.topk_idx, dc.topk_w)
-        if ev is not None:
-            ev[1].record(stream)
-        moe.demand_hist(dc.topk_idx, cfg.E, dc.counts)
-        if ev is not None:
-            ev[2].record(stream)
-        moe.replica_assign(dc.counts, dc.replica_offsets, dc.replica_slots, dc.slot_rank, cfg.R,
-                           dc.expert_slot, dc.expert_rank, dc.rank_active)
-        if ev is not None:
-            ev[3].record(stream)
-        moe.build_layout(dc.topk_idx, dc.topk_w, dc.expert_rank, dc.layout)
-        if ev is not None:
-            ev[4].record(stream)
+        marks = iter(ev) if ev is not None else None
+
+        def mark():
+            if marks is not None:
+                next(marks).record(stream)
+
+        mark()
+        if args.fused:
+            dc.route_single_replica(logits, static_rank)
+            mark()
+        else:
+            moe.route_topk(logits, cfg.k, cfg.n_groups, cfg.groups_per_token, False, dc.topk_idx, dc.topk_w)
+            mark()
+            moe.demand_hist(dc.topk_idx, cfg.E, dc.counts)
+            mark()
+            moe.replica_assign(dc.counts, dc.replica_offsets, dc.replica_slots, dc.slot_rank, cfg.R,
+                               dc.expert_slot, dc.expert_rank, dc.rank_active)
+            mark()
+            moe.build_layout(dc.topk_idx, dc.topk_w, dc.expert_rank, dc.layout)
+            mark()
         moe.pack(x, dc.layout, dc.packed, dc.packed_hop1)
-        if ev is not None:
-            ev[5].record(stream)
+        mark()
         dc.combine()
-        if ev is not None:
-            ev[6].record(stream)
+        mark()
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -217,7 +228,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     rows1 = int(dc.layout.num_rows_hop1.item()) if cfg.mode == W.TWO_HOP else 0
 
     # device-resident timed region: CUDA events on the launching stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     barrier()
     launches0 = moe.kernel_launches()
     t_start = torch.cuda.Event(enable_timing=True)
@@ -234,6 +245,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     st = moe.get_status()
     if st != 0:
         raise RuntimeError(f"device status after timing: {moe.status_string(st)}")
+    eager_ms = elapsed_ms
+    if args.graph:
+        # the same step captured once in a CUDA graph and replayed: no host
+        # launch latency between the kernels (the decode workloads' regime)
+        g = torch.cuda.CUDAGraph()
+        n0 = moe.kernel_launches()
+        with torch.cuda.graph(g):
+            one_step()
+        kernels_per_step = moe.kernel_launches() - n0
+        for _ in range(args.warmup):
+            g.replay()
+        barrier()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        g1.record(stream)
+        barrier()
+        elapsed_ms = g0.elapsed_time(g1)
+        launches = kernels_per_step * args.steps
+        st = moe.get_status()
+        if st != 0:
+            raise RuntimeError(f"device status after graph replays: {moe.status_string(st)}")
+        del g
 
     # end to end through the public API: pinned host inputs in, result out
     out_h = torch.empty((cfg.T, cfg.H), dtype=tdt).pin_memory()
@@ -257,6 +293,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if st != 0:
         raise RuntimeError(f"device status after e2e: {moe.status_string(st)}")
 
+    # workload statistics of the last pass (device kernels, outside the timed regions)
+    stats = moe.dispatch_stats(dc.counts, dc.layout.send_counts).cpu().tolist()
+    _, tb_active = moe.token_balanced_assign(dc.counts, dc.replica_offsets, dc.replica_slots,
+                                             dc.slot_rank, cfg.R)
+    workload_stats = dict(zip(moe.STAT_NAMES, stats))
+    workload_stats.update(
+        max_active_metro=int(dc.rank_active.max().item()),
+        max_active_token_balanced=int(tb_active.max().item()),
+        active_experts=int((dc.counts > 0).sum().item()))
+    st = moe.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status after statistics: {moe.status_string(st)}")
+
     # whole-job aggregation: max time over ranks, rows summed over ranks
     agg = aggregate(dist, dev, [elapsed_ms, e2e_ms], [rows * args.steps, rows * e2e_steps])
     if dist is not None:
@@ -266,7 +315,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     (elapsed_max, e2e_max), (rows_all, rows_e2e_all) = agg
     peak, peak_kind = measured_peak()
     bytes_ = step_bytes(cfg, rows, rows1, rm.S)
-    step_total = sum(bytes_.values())
+    step_total = sum(bytes_[n] for n in names)
     ms_step = elapsed_max / args.steps
     dom = max(("pack", "combine"), key=lambda n: per[n])
     achieved = bytes_[dom] / (per[dom] * 1e-3) / 1e9
@@ -294,7 +343,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "l2": "inputs larger than L2 (activations %.2f GB, packed rows %.2f GB per step; L2 126 MB)"
                   % (cfg.T * cfg.H * cfg.elem_bytes / 1e9, rows * cfg.H * cfg.elem_bytes / 1e9),
             "parallelism": f"independent replica per GPU x{world}",
+            "launch": "cuda_graph" if args.graph else "eager",
+            "front_end": "fused single-replica route+layout" if args.fused else "separate calls",
         },
+        "eager_ms_per_step": eager_ms / args.steps,
         "hbm_GBps": step_total / (ms_step * 1e-3) / 1e9,
         "hbm_frac_of_measured": step_total / (ms_step * 1e-3) / 1e9 / peak,
         "hbm_frac_of_8TBps": step_total / (ms_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
@@ -310,6 +362,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "steps": e2e_steps, "ms_per_step": e2e_max / e2e_steps},
         "gpu_launches": int(launches),
         "clocks": clocks,
+        "workload_stats": workload_stats,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args)
@@ -417,6 +470,11 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-tokens", type=int, default=8192)
     ap.add_argument("--ref-sample-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="route, histogram, assignment and layout in one fused pass "
+                         "(placements with one replica per expert)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of the step captured in a CUDA graph")
     args = ap.parse_args(argv)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -63,6 +63,11 @@ _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_debug_set_wait": (ctypes.c_int, [ctypes.c_uint64, _I]),
     "moe_kernel_launches": (ctypes.c_uint64, []),
+    "moe_route_layout_single_replica": (ctypes.c_int, [_P, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _I,
+                                                       _P, _P, _P, _P, ctypes.POINTER(moe_layout),
+                                                       _P, _SZ, _S]),
+    "moe_dispatch_stats": (ctypes.c_int, [_P, _I, _P, _I, _P, _S]),
+    "moe_token_balanced_assign": (ctypes.c_int, [_P, _I, _P, _P, _I, _P, _I, _I, _P, _P, _S]),
 }
 
 
@@ -273,3 +278,60 @@ def combine(y: torch.Tensor, layout: Layout, out=None, out_dtype=None, row_coef=
     _check(lib().moe_combine(_p(y), _DT[y.dtype], H, ctypes.byref(L.struct), _p(row_coef), _p(out),
                              _DT[out_dtype], _p(hop1_buf), _stream(stream)), "moe_combine")
     return out
+
+
+# ------------------------------------------------------------- statistics ----
+STAT_NAMES = ("expert_max_mean", "rank_gini", "rank_max_mean", "own_rank_row_share")
+
+
+def dispatch_stats(counts: torch.Tensor, send_counts: torch.Tensor, out=None, stream=None):
+    """The four statistics as a float64 device tensor [4] (see STAT_NAMES)."""
+    _need(counts, torch.int32, "counts", 1)
+    _need(send_counts, torch.int32, "send_counts")
+    R = int(round(send_counts.numel() ** 0.5))
+    if R * R != send_counts.numel():
+        raise ValueError("send_counts must be R x R")
+    out = torch.empty(4, dtype=torch.float64, device=counts.device) if out is None else out
+    _need(out, torch.float64, "out", 1)
+    _check(lib().moe_dispatch_stats(_p(counts), counts.numel(), _p(send_counts), R, _p(out),
+                                    _stream(stream)), "moe_dispatch_stats")
+    return out
+
+
+def token_balanced_assign(counts, replica_offsets, replica_slots, slot_rank, R: int,
+                          slot_tokens=None, rank_active=None, stream=None):
+    for t, n in ((counts, "counts"), (replica_offsets, "replica_offsets"),
+                 (replica_slots, "replica_slots"), (slot_rank, "slot_rank")):
+        _need(t, torch.int32, n, 1)
+    S = slot_rank.numel()
+    dev = counts.device
+    slot_tokens = torch.empty(S, dtype=torch.int32, device=dev) if slot_tokens is None else slot_tokens
+    rank_active = torch.empty(R, dtype=torch.int32, device=dev) if rank_active is None else rank_active
+    _check(lib().moe_token_balanced_assign(_p(counts), counts.numel(), _p(replica_offsets),
+                                           _p(replica_slots), replica_slots.numel(), _p(slot_rank), S, R,
+                                           _p(slot_tokens), _p(rank_active), _stream(stream)),
+           "moe_token_balanced_assign")
+    return slot_tokens, rank_active
+
+
+def route_layout_single_replica(logits: torch.Tensor, k: int, expert_rank: torch.Tensor, layout: Layout,
+                                n_groups: int = 0, groups_per_token: int = 0, renormalize: bool = False,
+                                topk_idx=None, topk_w=None, counts=None, rank_active=None, stream=None):
+    """route_topk + demand_hist + replica_assign + build_layout in one pass for
+    placements with one replica per expert (expert_rank: that replica's rank)."""
+    _need(logits, torch.float32, "logits", 2)
+    _need(expert_rank, torch.int32, "expert_rank", 1)
+    T, E = logits.shape
+    L = layout
+    if (T, k, E) != (L.T, L.k, L.E):
+        raise ValueError("logits / k do not match the layout's sizes")
+    dev = logits.device
+    topk_idx = torch.empty((T, k), dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
+    topk_w = torch.empty((T, k), dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    counts = torch.empty(E, dtype=torch.int32, device=dev) if counts is None else counts
+    _check(lib().moe_route_layout_single_replica(
+        _p(logits), T, E, k, n_groups, groups_per_token, int(renormalize), _p(expert_rank),
+        L.tokens_per_rank, L.R, L.ranks_per_group, L.mode, _p(topk_idx), _p(topk_w), _p(counts),
+        _p(rank_active), ctypes.byref(L.struct), _p(L.workspace), L.workspace.numel(), _stream(stream)),
+        "moe_route_layout_single_replica")
+    return topk_idx, topk_w, counts

@@ -24,30 +24,12 @@
 // present in the warp, then each lane walks its own bits.  Experts (PER_PICK,
 // up to 1024 bins) are merged instead: each round takes the smallest key
 // (rank << 10 | expert) left in the warp with redux.sync.min.
-#include "moe_internal.cuh"
+#include "layout_common.cuh"
 
 namespace moe {
+namespace layout {
 namespace {
 
-constexpr int kTile = 256;  // tokens per tile, one per thread
-constexpr int kWarps = kTile / 32;
-constexpr int kMaxBins = kMaxE;  // >= max(E, R + G)
-constexpr int kSendSmem = kMaxR * kMaxR;
-constexpr unsigned kFull = 0xffffffffu;
-constexpr unsigned long long kFlagAgg = 1ull << 32;
-constexpr unsigned long long kFlagInc = 2ull << 32;
-
-struct LayoutArgs {
-  const int *idx;
-  const float *w;
-  const int *expert_rank;
-  int T, tpr, k, E, R, rpg, G, mode, NB, num_tiles;
-  int *counters;  // [0] place-kernel ticket, [1] count-kernel blocks done
-  int *totals;    // [NB]
-  int *seg_off;   // [NB]
-  unsigned long long *state;  // [num_tiles][NB]: flag << 32 | count
-  moe_layout L;
-};
 
 // One token's picks as seen by one thread.
 template <int KM>
@@ -140,89 +122,6 @@ __device__ __forceinline__ void warp_merge(const TokenPicks<KM> &p, int rpg, F &
   }
 }
 
-__device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
-  const unsigned lo = __reduce_or_sync(kFull, (unsigned)m);
-  const unsigned hi = __reduce_or_sync(kFull, (unsigned)(m >> 32));
-  return ((unsigned long long)hi << 32) | lo;
-}
-
-// Bins given as 64-bit masks (ranks, or groups): for every bin present in the
-// warp, f(bin, has, ball) runs on all lanes with the warp's ballot of the bin.
-template <class F>
-__device__ __forceinline__ void warp_mask_bins(unsigned long long mask, F &&f) {
-  unsigned long long wm = warp_or64(mask);
-  while (wm) {
-    const int b = __ffsll((long long)wm) - 1;
-    wm &= wm - 1;
-    const bool has = (mask >> b) & 1ull;
-    f(b, has, __ballot_sync(kFull, has));
-  }
-}
-
-__device__ __forceinline__ unsigned lanemask_lt() {
-  unsigned m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
-__device__ __forceinline__ unsigned long long group_bits(int g, int rpg) {
-  const unsigned long long ones = (rpg >= 64) ? ~0ull : ((1ull << rpg) - 1ull);
-  return (rpg >= 64) ? ones : (ones << (g * rpg));
-}
-
-// ------------------------------------------------------------- finalize ----
-// Runs in the last count block, all threads: the totals are loaded into
-// shared memory in parallel (tot), then thread 0 scans them into segment
-// offsets and the host-visible offsets.
-__device__ void finalize(const LayoutArgs &a, const int *s_er, int *tot, DeviceCtx ctx) {
-  for (int i = threadIdx.x; i < a.NB; i += blockDim.x) tot[i] = __ldcg(a.totals + i);
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  const moe_layout &L = a.L;
-  if (a.mode == MOE_LAYOUT_PER_PICK) {
-    int base[kMaxR + 1];
-    for (int r = 0; r <= a.R; ++r) base[r] = 0;
-    for (int e = 0; e < a.E; ++e) {
-      const int r = s_er[e];
-      if ((unsigned)r < (unsigned)a.R) base[r + 1] += tot[e];
-    }
-    for (int r = 0; r < a.R; ++r) base[r + 1] += base[r];
-    for (int r = 0; r <= a.R; ++r) L.rank_offsets[r] = base[r];
-    const int n = base[a.R];
-    for (int e = 0; e < a.E; ++e) {
-      const int r = s_er[e];
-      if ((unsigned)r < (unsigned)a.R) {
-        a.seg_off[e] = base[r];
-        base[r] += tot[e];
-      } else {
-        a.seg_off[e] = 0;
-      }
-    }
-    *L.num_rows = n;
-    if (n > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
-    return;
-  }
-  int run = 0;
-  for (int r = 0; r < a.R; ++r) {
-    a.seg_off[r] = run;
-    L.rank_offsets[r] = run;
-    run += tot[r];
-  }
-  L.rank_offsets[a.R] = run;
-  *L.num_rows = run;
-  if (run > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
-  if (a.mode == MOE_LAYOUT_TWO_HOP) {
-    int run1 = 0;
-    for (int g = 0; g < a.G; ++g) {
-      a.seg_off[a.R + g] = run1;
-      L.group_offsets[g] = run1;
-      run1 += tot[a.R + g];
-    }
-    L.group_offsets[a.G] = run1;
-    *L.num_rows_hop1 = run1;
-    if (run1 > L.capacity_hop1) set_status(ctx.status, MOE_ERR_CAPACITY);
-  }
-}
 
 // ---------------------------------------------------------------- count ----
 template <int KM>
@@ -478,7 +377,7 @@ __global__ void __launch_bounds__(kTile) layout_place_kernel(LayoutArgs a, Devic
 }
 
 template <int KM>
-cudaError_t launch_km(const LayoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+cudaError_t launch_count_place(const LayoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   layout_count_kernel<KM><<<a.num_tiles, kTile, 0, s>>>(a, ctx);
   cudaError_t err = count_launch(cudaGetLastError());
   if (err != cudaSuccess) return err;
@@ -486,39 +385,17 @@ cudaError_t launch_km(const LayoutArgs &a, const DeviceCtx &ctx, cudaStream_t s)
   return count_launch(cudaGetLastError());
 }
 
-int num_bins(int E, int R, int rpg, int mode) {
-  if (mode == MOE_LAYOUT_PER_PICK) return E;
-  if (mode == MOE_LAYOUT_TWO_HOP) return R + R / rpg;
-  return R;
+template <int KM>
+cudaError_t launch_place(const LayoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+  layout_place_kernel<KM><<<a.num_tiles, kTile, 0, s>>>(a, ctx);
+  return count_launch(cudaGetLastError());
 }
-
-size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 }  // namespace
 
-size_t layout_workspace_bytes(int T, int k, int E, int R, int rpg, int mode) {
-  (void)k;
-  const int NB = num_bins(E, R, rpg, mode);
-  const size_t tiles = (size_t)((T + kTile - 1) / kTile);
-  return align16(sizeof(int) * (2 + 2 * (size_t)NB)) + tiles * NB * sizeof(unsigned long long);
-}
-
-cudaError_t launch_build_layout(const int *idx, const float *w, const int *expert_rank, int T,
-                                int tokens_per_rank, int k, int E, int R, int rpg, int mode,
-                                const moe_layout &L, void *ws, const DeviceCtx &ctx,
-                                cudaStream_t s) {
-  cudaError_t err;
-  if (T == 0) {
-    if ((err = cudaMemsetAsync(L.rank_offsets, 0, sizeof(int) * (R + 1), s)) != cudaSuccess) return err;
-    if ((err = cudaMemsetAsync(L.num_rows, 0, sizeof(int), s)) != cudaSuccess) return err;
-    if ((err = cudaMemsetAsync(L.send_counts, 0, sizeof(int) * R * R, s)) != cudaSuccess) return err;
-    if (mode == MOE_LAYOUT_TWO_HOP) {
-      if ((err = cudaMemsetAsync(L.group_offsets, 0, sizeof(int) * (R / rpg + 1), s)) != cudaSuccess)
-        return err;
-      if ((err = cudaMemsetAsync(L.num_rows_hop1, 0, sizeof(int), s)) != cudaSuccess) return err;
-    }
-    return cudaSuccess;
-  }
+LayoutArgs make_layout_args(const int *idx, const float *w, const int *expert_rank, int T,
+                            int tokens_per_rank, int k, int E, int R, int rpg, int mode,
+                            const moe_layout &L, void *ws) {
   LayoutArgs a;
   a.idx = idx;
   a.w = w;
@@ -539,12 +416,57 @@ cudaError_t launch_build_layout(const int *idx, const float *w, const int *exper
   a.seg_off = a.totals + a.NB;
   a.state = reinterpret_cast<unsigned long long *>(base + align16(sizeof(int) * (2 + 2 * (size_t)a.NB)));
   a.L = L;
-  if ((err = cudaMemsetAsync(a.counters, 0, sizeof(int) * (2 + (size_t)a.NB), s)) != cudaSuccess) return err;
-  if ((err = cudaMemsetAsync(L.send_counts, 0, sizeof(int) * (size_t)R * R, s)) != cudaSuccess) return err;
-  if (k <= 2) return launch_km<2>(a, ctx, s);
-  if (k <= 4) return launch_km<4>(a, ctx, s);
-  if (k <= 8) return launch_km<8>(a, ctx, s);
-  return launch_km<16>(a, ctx, s);
+  return a;
+}
+
+cudaError_t layout_clear(const LayoutArgs &a, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(a.counters, 0, sizeof(int) * (2 + (size_t)a.NB), s);
+  if (err != cudaSuccess) return err;
+  return cudaMemsetAsync(a.L.send_counts, 0, sizeof(int) * (size_t)a.R * a.R, s);
+}
+
+cudaError_t layout_empty(const moe_layout &L, int R, int rpg, int mode, cudaStream_t s) {
+  cudaError_t err;
+  if ((err = cudaMemsetAsync(L.rank_offsets, 0, sizeof(int) * (R + 1), s)) != cudaSuccess) return err;
+  if ((err = cudaMemsetAsync(L.num_rows, 0, sizeof(int), s)) != cudaSuccess) return err;
+  if ((err = cudaMemsetAsync(L.send_counts, 0, sizeof(int) * R * R, s)) != cudaSuccess) return err;
+  if (mode == MOE_LAYOUT_TWO_HOP) {
+    if ((err = cudaMemsetAsync(L.group_offsets, 0, sizeof(int) * (R / rpg + 1), s)) != cudaSuccess)
+      return err;
+    if ((err = cudaMemsetAsync(L.num_rows_hop1, 0, sizeof(int), s)) != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_layout_place(const LayoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+  if (a.k <= 2) return launch_place<2>(a, ctx, s);
+  if (a.k <= 4) return launch_place<4>(a, ctx, s);
+  if (a.k <= 8) return launch_place<8>(a, ctx, s);
+  return launch_place<16>(a, ctx, s);
+}
+
+}  // namespace layout
+
+size_t layout_workspace_bytes(int T, int k, int E, int R, int rpg, int mode) {
+  (void)k;
+  const int NB = layout::num_bins(E, R, rpg, mode);
+  const size_t tiles = (size_t)((T + layout::kTile - 1) / layout::kTile);
+  return layout::align16(sizeof(int) * (2 + 2 * (size_t)NB)) + tiles * NB * sizeof(unsigned long long);
+}
+
+cudaError_t launch_build_layout(const int *idx, const float *w, const int *expert_rank, int T,
+                                int tokens_per_rank, int k, int E, int R, int rpg, int mode,
+                                const moe_layout &L, void *ws, const DeviceCtx &ctx,
+                                cudaStream_t s) {
+  if (T == 0) return layout::layout_empty(L, R, rpg, mode, s);
+  const layout::LayoutArgs a =
+      layout::make_layout_args(idx, w, expert_rank, T, tokens_per_rank, k, E, R, rpg, mode, L, ws);
+  cudaError_t err = layout::layout_clear(a, s);
+  if (err != cudaSuccess) return err;
+  if (k <= 2) return layout::launch_count_place<2>(a, ctx, s);
+  if (k <= 4) return layout::launch_count_place<4>(a, ctx, s);
+  if (k <= 8) return layout::launch_count_place<8>(a, ctx, s);
+  return layout::launch_count_place<16>(a, ctx, s);
 }
 
 }  // namespace moe

@@ -110,6 +110,18 @@ cudaError_t launch_build_layout(const int *idx, const float *w, const int *exper
                                 cudaStream_t s);
 cudaError_t launch_pack(const void *x, int elem_bytes, int H, const moe_layout &L, void *packed,
                         void *packed_hop1, const DeviceCtx &ctx, cudaStream_t s);
+cudaError_t launch_route_layout_static(const float *logits, int T, int E, int k, int n_groups,
+                                       int gpt, int renorm, const int *expert_rank,
+                                       int tokens_per_rank, int R, int rpg, int mode, int *idx,
+                                       float *w, int *counts, int *rank_active,
+                                       const moe_layout &L, void *ws, const DeviceCtx &ctx,
+                                       cudaStream_t s);
+cudaError_t launch_dispatch_stats(const int *counts, int E, const int *send_counts, int R,
+                                  double *stats, const DeviceCtx &ctx, cudaStream_t s);
+cudaError_t launch_token_balanced(const int *counts, int E, const int *off, const int *slots,
+                                  int n_entries, const int *slot_rank, int S, int R,
+                                  int *slot_tokens, int *rank_active, const DeviceCtx &ctx,
+                                  cudaStream_t s);
 cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
                            const float *row_coef, void *out, int out_dtype, void *hop1_buf,
                            const DeviceCtx &ctx, cudaStream_t s);

@@ -53,6 +53,13 @@ class DispatchCombine:
                          self.R, self.expert_slot, self.expert_rank, self.rank_active)
         B.build_layout(self.topk_idx, self.topk_w, self.expert_rank, self.layout)
 
+    def route_single_replica(self, logits: torch.Tensor, expert_rank: torch.Tensor):
+        """The same outputs as route() for a map with one replica per expert,
+        in one fused pass (expert_rank: each expert's only rank)."""
+        B.route_layout_single_replica(logits, self.k, expert_rank, self.layout, self.n_groups,
+                                      self.groups_per_token, self.renormalize, self.topk_idx,
+                                      self.topk_w, self.counts, self.rank_active)
+
     def dispatch(self, logits: torch.Tensor, x: torch.Tensor) -> torch.Tensor:
         self.route(logits)
         B.pack(x, self.layout, self.packed, self.packed_hop1)

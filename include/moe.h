@@ -246,6 +246,58 @@ MOE_API int moe_combine(const void *y, int32_t dtype, int32_t H, const moe_layou
                 moe_stream_t stream);
 
 /*
+ * moe_route_topk, moe_demand_hist, moe_replica_assign and moe_build_layout in
+ * one pass, for placements with exactly one replica per expert.  Source: with
+ * a single replica, the METRO assignment of "METRO AllGather vs AllToAll for
+ * MoE decode" (sections "changes the routing information" and "Add the
+ * expert-weight traffic term") has no choice to make, so each pick's
+ * destination rank is known as soon as the pick is; one kernel routes the
+ * tokens and counts the demand vector, the layout's bins and the send matrix,
+ * and the layout's place kernel follows.  Every output equals that of the
+ * separate calls.
+ * expert_rank [E]: rank of each expert's only replica (every entry in [0, R);
+ * a pick of an expert outside it sets MOE_ERR_BAD_INPUT and is skipped).
+ * counts [E] out: the demand vector.  rank_active [R] out, or NULL: activated
+ * experts per rank.  topk_idx, topk_w, the layout and the workspace as in
+ * moe_route_topk and moe_build_layout.
+ */
+MOE_API int moe_route_layout_single_replica(
+    const float *logits, int32_t T, int32_t E, int32_t k, int32_t n_groups,
+    int32_t groups_per_token, int32_t renormalize, const int32_t *expert_rank,
+    int32_t tokens_per_rank, int32_t R, int32_t ranks_per_group, int32_t mode, int32_t *topk_idx,
+    float *topk_w, int32_t *counts, int32_t *rank_active, moe_layout *layout, void *workspace,
+    size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * Statistics of one dispatch (one CTA).  Source: gist.science summary of
+ * DODOCO, "Methodology": the per-expert max/mean ratio measures routing skew
+ * independent of the expert-to-rank map; the Gini coefficient measures
+ * per-rank load imbalance.  Per-rank load = rows each destination rank
+ * receives (column sums of send_counts).
+ * counts [E] (demand vector), send_counts [R*R] (from moe_build_layout).
+ * stats [4] float64 out: per-expert max/mean, Gini of the per-rank load
+ * (sum over ordered pairs |x_i - x_j| / (2 R^2 mean)), per-rank max/mean, and
+ * the share of rows that stay on their source rank; 0 when there is no load.
+ */
+MOE_API int moe_dispatch_stats(const int32_t *counts, int32_t E, const int32_t *send_counts,
+                               int32_t R, double *stats, moe_stream_t stream);
+
+/*
+ * Token-balanced replica routing, the comparison policy of "METRO AllGather vs
+ * AllToAll for MoE decode" (sections "Add the expert-weight traffic term" and
+ * "Know what the paper actually measured": EPLB token routing).  Each
+ * expert's c tokens are dealt round-robin over its n valid replicas in
+ * ascending slot id: the i-th gets floor(c / n) + (i < c mod n) tokens.  A
+ * replica with a token is activated.  Map arguments as moe_replica_assign.
+ * slot_tokens [S] out (0 for slots of inactive experts), rank_active [R] out.
+ */
+MOE_API int moe_token_balanced_assign(const int32_t *counts, int32_t E,
+                                      const int32_t *replica_offsets, const int32_t *replica_slots,
+                                      int32_t n_replica_entries, const int32_t *slot_rank, int32_t S,
+                                      int32_t R, int32_t *slot_tokens, int32_t *rank_active,
+                                      moe_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device (MOE_OK if no device-side error was recorded since the last
  * call).  The word is shared by every stream on the device.
