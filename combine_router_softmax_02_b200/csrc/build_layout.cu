@@ -15,10 +15,11 @@
 //   seg_off[bin] + (rows of bin in earlier tiles) + (rows of bin in earlier
 //   warps of the tile) + (rows of bin in earlier lanes of the warp).
 // Kernel 1 (count) builds the per-bin totals with block histograms and global
-// atomics; its last block turns them into segment offsets.  Kernel 2 (place)
-// takes tiles in ticket order, publishes each tile's per-bin aggregate, looks
-// back over its predecessors for the exclusive prefix (bounded waits), and
-// writes the rows.  Within a warp a bin's ballot over the lanes gives both its
+// atomics, and publishes each tile's per-bin aggregate as a look-back flag;
+// its last block turns the totals into segment offsets.  Kernel 2 (place)
+// takes tiles in ticket order, looks back over its predecessors' flags for the
+// exclusive prefix (16 flags per round, bounded waits), publishes its
+// inclusive prefix, and writes the rows.  Within a warp a bin's ballot over the lanes gives both its
 // count and each lane's position in token order (stability).  Ranks and
 // groups (at most 64 each) are 64-bit masks per token: one ballot per bin
 // present in the warp, then each lane walks its own bits.  Experts (PER_PICK,
@@ -134,10 +135,7 @@ __global__ void __launch_bounds__(kTile) layout_count_kernel(LayoutArgs a, Devic
   const int tid = threadIdx.x, lane = tid & 31;
   const int t = tile * kTile + tid;
   for (int i = tid; i < a.E; i += kTile) s_er[i] = a.expert_rank[i];
-  for (int i = tid; i < a.NB; i += kTile) {
-    s_cnt[i] = 0;
-    a.state[(size_t)tile * a.NB + i] = 0ull;  // the place kernel's flags start clear
-  }
+  for (int i = tid; i < a.NB; i += kTile) s_cnt[i] = 0;
   // source ranks are < R, so the block's send-count matrix fits R*R <= 4096 entries
   for (int i = tid; i < a.R * a.R; i += kTile) s_send[i] = 0;
   __syncthreads();
@@ -181,6 +179,12 @@ __global__ void __launch_bounds__(kTile) layout_count_kernel(LayoutArgs a, Devic
   }
   if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
   __syncthreads();
+  // publish this tile's aggregates for the place kernel's look-back (the
+  // first tile's is its inclusive prefix); a silent tile leaves its flags clear
+  const bool silent = (tile == ctx.silent_tile);
+  for (int i = tid; i < a.NB; i += kTile)
+    a.state[(size_t)tile * a.NB + i] =
+        silent ? 0ull : ((tile == 0 ? kFlagInc : kFlagAgg) | (unsigned)s_cnt[i]);
   for (int i = tid; i < a.NB; i += kTile)
     if (s_cnt[i]) atomicAdd(&a.totals[i], s_cnt[i]);
   for (int i = tid; i < a.R * a.R; i += kTile)
@@ -210,6 +214,31 @@ __device__ __forceinline__ unsigned long long wait_published(const unsigned long
       return kFlagInc;  // treat as an inclusive zero so the chain ends
     }
   }
+}
+
+constexpr int kWindow = 16;
+
+// Exclusive prefix of one bin before `tile`: the bin's flags of the earlier
+// tiles are summed from tile - 1 backwards until an inclusive prefix is met,
+// kWindow predecessors per round with all of their loads in flight.
+__device__ __forceinline__ int look_back(const unsigned long long *col, int NB, int tile,
+                                         const DeviceCtx &ctx, bool &timed_out) {
+  int excl = 0;
+  for (int q = tile - 1; q >= 0; q -= kWindow) {
+    unsigned long long v[kWindow];
+#pragma unroll
+    for (int i = 0; i < kWindow; ++i)
+      v[i] = (q - i >= 0) ? ld_acquire_u64(col + (size_t)(q - i) * NB) : 0ull;
+#pragma unroll
+    for (int i = 0; i < kWindow; ++i) {
+      if (q - i < 0) return excl;
+      unsigned long long w = v[i];
+      if ((w >> 32) == 0ull) w = wait_published(col + (size_t)(q - i) * NB, ctx, timed_out);
+      excl += (int)(unsigned)(w & 0xffffffffull);
+      if ((w >> 32) == 2ull) return excl;
+    }
+  }
+  return excl;
 }
 
 template <int KM>
@@ -279,11 +308,7 @@ __global__ void __launch_bounds__(kTile) layout_place_kernel(LayoutArgs a, Devic
       if (!silent) st_release_u64(mine, kFlagInc | (unsigned)agg);
     } else {
       if (!silent) st_release_u64(mine, kFlagAgg | (unsigned)agg);
-      for (int q = tile - 1; q >= 0; --q) {
-        const unsigned long long v = wait_published(a.state + (size_t)q * a.NB + b, ctx, timed_out);
-        excl += (int)(unsigned)(v & 0xffffffffull);
-        if ((v >> 32) == 2ull) break;
-      }
+      excl = look_back(a.state + b, a.NB, tile, ctx, timed_out);
       if (!silent) st_release_u64(mine, kFlagInc | (unsigned)(excl + agg));
     }
     s_base[b] = __ldcg(a.seg_off + b) + excl;

@@ -395,6 +395,68 @@ def check_round_to(round_to):
     assert round_to(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8]), "bf16").tolist() == [1.0, 1 + 2.0 ** -6]
 
 
+# ------------------------------------------------------------- placement ----
+def check_coselection(coselection):
+    rng = np.random.default_rng(14)
+    for T, E, k in [(1, 4, 2), (40, 8, 3), (200, 16, 5)]:
+        idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
+        C = coselection(idx, E)
+        ref = collections.Counter()
+        for t in range(T):
+            for a in idx[t]:
+                for b in idx[t]:
+                    if a != b:
+                        ref[int(a), int(b)] += 1
+        assert all(C[a][b] == ref.get((a, b), 0) for a in range(E) for b in range(E))
+        assert np.array_equal(C, C.T) and not np.diag(C).any()
+        assert int(C.sum()) == T * k * (k - 1)               # every ordered pair of distinct picks
+
+
+def brute_best_within(C, R):
+    """The largest total within-rank co-selection over every balanced placement (tiny E)."""
+    import itertools
+    E = C.shape[0]
+    cap = E // R
+    best = -1
+    for labels in itertools.product(range(R), repeat=E):
+        if any(labels.count(r) != cap for r in range(R)):
+            continue
+        s = sum(C[a][b] for a in range(E) for b in range(E) if a < b and labels[a] == labels[b])
+        best = max(best, s)
+    return best
+
+
+def check_placement(correlated_placement):
+    # no co-selection at all: consecutive blocks of the demand order
+    counts = np.array([5, 9, 9, 1, 7, 3])
+    rank = correlated_placement(np.zeros((6, 6), np.int64), counts, 3)
+    order = sorted(range(6), key=lambda e: (-counts[e], e))            # 1, 2, 4, 0, 5, 3
+    assert [int(rank[e]) for e in order] == [0, 0, 1, 1, 2, 2]
+    # hand-worked: seed 0 (demand 9) pulls 3 (co-selection 4); seed 1 pulls 2
+    C = np.array([[0, 1, 0, 4], [1, 0, 2, 0], [0, 2, 0, 1], [4, 0, 1, 0]])
+    assert correlated_placement(C, np.array([9, 8, 1, 1]), 2).tolist() == [0, 1, 1, 0]
+    # planted clusters: every cluster lands on one rank
+    rng = np.random.default_rng(15)
+    for E, R in [(16, 4), (64, 32), (24, 8)]:
+        perm = rng.permutation(E)
+        cl = np.empty(E, np.int64)
+        cl[perm] = np.arange(E) // (E // R)
+        C = np.where(cl[:, None] == cl[None, :], 50, 1) - np.eye(E, dtype=np.int64) * 50
+        rank = correlated_placement(C, rng.integers(1, 100, size=E), R)
+        assert np.bincount(rank, minlength=R).tolist() == [E // R] * R
+        for c in range(R):
+            assert len(set(rank[cl == c].tolist())) == 1
+    # tiny instances: balanced, and never better than the brute-force optimum
+    for _ in range(12):
+        E, R = 6, int(rng.choice([2, 3]))
+        A = rng.integers(0, 6, size=(E, E))
+        C = np.triu(A, 1) + np.triu(A, 1).T
+        rank = correlated_placement(C, rng.integers(0, 9, size=E), R)
+        assert np.bincount(rank, minlength=R).tolist() == [E // R] * R
+        got = sum(C[a][b] for a in range(E) for b in range(E) if a < b and rank[a] == rank[b])
+        assert got <= brute_best_within(C, R)
+
+
 # ----------------------------------------------------------- statistics ----
 def check_gini(gini):
     assert gini([3, 3, 3, 3]) == 0.0 and gini([0, 0]) == 0.0

@@ -169,3 +169,10 @@ def test_token_balanced_listed_order_caught():
         return st, act
     with pytest.raises(AssertionError):
         pins.check_token_balanced(mutant)
+
+
+def test_placement_ignoring_affinity_caught():
+    def mutant(C, counts, R):
+        return oracle.correlated_placement(np.zeros_like(C), counts, R)
+    with pytest.raises(AssertionError):
+        pins.check_placement(mutant)

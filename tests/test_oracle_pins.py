@@ -100,3 +100,27 @@ def test_uniform_own_row_share_single_pick():
     L = oracle.build_layout(idx, w, W.expert_home_rank(cfg), cfg.T // 8, 8, oracle.DEDUP)
     share = oracle.dispatch_stats(oracle.demand_hist(idx, cfg.E), L["send_counts"])["own_rank_row_share"]
     assert abs(share - 0.125) < 5 * (0.125 * 0.875 / cfg.T) ** 0.5
+
+
+def test_coselection_brute_force():
+    pins.check_coselection(oracle.coselection)
+
+
+def test_correlated_placement_closed_forms_and_brute_force():
+    pins.check_placement(oracle.correlated_placement)
+
+
+def test_derived_placement_shrinks_dedup_rows():
+    """On the clustered training workload, the placement derived from the
+    co-selection counts sends fewer dedup rows than round-robin placement
+    (the direction of the summary's 'removes up to 58% of dispatched rows')."""
+    import workloads as W
+    cfg = W.CONFIGS["c3"]
+    idx, w = oracle.route_topk(W.make_logits(cfg, 0), cfg.k)
+    er = oracle.correlated_placement(oracle.coselection(idx, cfg.E), oracle.demand_hist(idx, cfg.E), cfg.R)
+    rows = {}
+    for name, rank in (("derived", er), ("roundrobin", W.expert_home_rank(cfg.with_(placement="roundrobin"))),
+                       ("block", W.expert_home_rank(cfg))):
+        rows[name] = int(oracle.build_layout(idx, w, rank, cfg.tokens_per_rank, cfg.R, oracle.DEDUP)["num_rows"])
+    assert rows["derived"] < rows["roundrobin"]
+    assert rows["derived"] <= 1.02 * rows["block"]      # close to the planted clusters
