@@ -66,6 +66,8 @@ _SIGS = {
     "moe_route_layout_single_replica": (ctypes.c_int, [_P, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _I,
                                                        _P, _P, _P, _P, ctypes.POINTER(moe_layout),
                                                        _P, _SZ, _S]),
+    "moe_coselection_hist": (ctypes.c_int, [_P, _I, _I, _I, _P, _S]),
+    "moe_correlated_placement": (ctypes.c_int, [_P, _P, _I, _I, _P, _S]),
     "moe_dispatch_stats": (ctypes.c_int, [_P, _I, _P, _I, _P, _S]),
     "moe_token_balanced_assign": (ctypes.c_int, [_P, _I, _P, _P, _I, _P, _I, _I, _P, _P, _S]),
 }
@@ -335,3 +337,23 @@ def route_layout_single_replica(logits: torch.Tensor, k: int, expert_rank: torch
         _p(rank_active), ctypes.byref(L.struct), _p(L.workspace), L.workspace.numel(), _stream(stream)),
         "moe_route_layout_single_replica")
     return topk_idx, topk_w, counts
+
+
+def coselection_hist(topk_idx: torch.Tensor, E: int, cosel=None, stream=None):
+    _need(topk_idx, torch.int32, "topk_idx", 2)
+    T, k = topk_idx.shape
+    cosel = torch.empty((E, E), dtype=torch.int32, device=topk_idx.device) if cosel is None else cosel
+    _need(cosel, torch.int32, "cosel")
+    _check(lib().moe_coselection_hist(_p(topk_idx), T, k, E, _p(cosel), _stream(stream)),
+           "moe_coselection_hist")
+    return cosel
+
+
+def correlated_placement(cosel: torch.Tensor, counts: torch.Tensor, R: int, expert_rank=None, stream=None):
+    _need(cosel, torch.int32, "cosel", 2)
+    _need(counts, torch.int32, "counts", 1)
+    E = counts.numel()
+    expert_rank = torch.empty(E, dtype=torch.int32, device=counts.device) if expert_rank is None else expert_rank
+    _check(lib().moe_correlated_placement(_p(cosel), _p(counts), E, R, _p(expert_rank), _stream(stream)),
+           "moe_correlated_placement")
+    return expert_rank

@@ -334,3 +334,29 @@ extern "C" int moe_route_layout_single_replica(
       ranks_per_group, mode, topk_idx, topk_w, counts, rank_active, L, workspace, ctx,
       reinterpret_cast<cudaStream_t>(stream)));
 }
+
+extern "C" {
+
+int moe_coselection_hist(const int32_t *topk_idx, int32_t T, int32_t k, int32_t E, int32_t *cosel,
+                         moe_stream_t stream) {
+  if (T < 0 || !valid_ekr(E, k) || !cosel || (T > 0 && !topk_idx)) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)T * k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  moe::DeviceCtx ctx;
+  int rc = get_ctx(&ctx);
+  if (rc) return rc;
+  return launched(moe::launch_coselection(topk_idx, T, k, E, cosel, ctx,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_correlated_placement(const int32_t *cosel, const int32_t *counts, int32_t E, int32_t R,
+                             int32_t *expert_rank, moe_stream_t stream) {
+  if (E < 1 || E > moe::kMaxE || R < 1 || R > moe::kMaxR || E % R != 0) return MOE_ERR_INVALID_ARG;
+  if (!cosel || !counts || !expert_rank) return MOE_ERR_INVALID_ARG;
+  moe::DeviceCtx ctx;
+  int rc = get_ctx(&ctx);
+  if (rc) return rc;
+  return launched(moe::launch_placement(cosel, counts, E, R, expert_rank, ctx,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

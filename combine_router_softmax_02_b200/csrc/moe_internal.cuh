@@ -116,6 +116,10 @@ cudaError_t launch_route_layout_static(const float *logits, int T, int E, int k,
                                        float *w, int *counts, int *rank_active,
                                        const moe_layout &L, void *ws, const DeviceCtx &ctx,
                                        cudaStream_t s);
+cudaError_t launch_coselection(const int *idx, int T, int k, int E, int *C, const DeviceCtx &ctx,
+                               cudaStream_t s);
+cudaError_t launch_placement(const int *C, const int *counts, int E, int R, int *expert_rank,
+                             const DeviceCtx &ctx, cudaStream_t s);
 cudaError_t launch_dispatch_stats(const int *counts, int E, const int *send_counts, int R,
                                   double *stats, const DeviceCtx &ctx, cudaStream_t s);
 cudaError_t launch_token_balanced(const int *counts, int E, const int *off, const int *slots,

@@ -269,6 +269,30 @@ MOE_API int moe_route_layout_single_replica(
     size_t workspace_bytes, moe_stream_t stream);
 
 /*
+ * Co-selection counts: cosel[e*E + f] = number of tokens whose picks include
+ * both e and f (e != f); symmetric, zero diagonal; zeroed by the call.
+ * Source: the ainewsletter summary of arXiv:2610.09372, "Correlations in
+ * router choices" (experts jointly selected by the same tokens).
+ * topk_idx [T][k] (distinct experts per token); cosel [E*E] int32 out.
+ */
+MOE_API int moe_coselection_hist(const int32_t *topk_idx, int32_t T, int32_t k, int32_t E,
+                                 int32_t *cosel, moe_stream_t stream);
+
+/*
+ * Correlated expert placement (one CTA).  Source: same summary, "Two locality
+ * techniques": experts often selected together go to the same GPU, so that a
+ * single-send dispatcher sends fewer rows.  The page gives no algorithm; this
+ * one grows the ranks one at a time, E/R experts each (R | E): the rank is
+ * seeded with the unplaced expert of highest demand, then takes the unplaced
+ * expert with the most co-selections with the rank's experts so far (ties:
+ * higher demand, then the lower id).
+ * cosel [E*E] symmetric (as moe_coselection_hist writes it), counts [E] (the
+ * demand vector), expert_rank [E] out: a placement with one replica per expert.
+ */
+MOE_API int moe_correlated_placement(const int32_t *cosel, const int32_t *counts, int32_t E,
+                                     int32_t R, int32_t *expert_rank, moe_stream_t stream);
+
+/*
  * Statistics of one dispatch (one CTA).  Source: gist.science summary of
  * DODOCO, "Methodology": the per-expert max/mean ratio measures routing skew
  * independent of the expert-to-rank map; the Gini coefficient measures
