@@ -93,15 +93,43 @@ __device__ __forceinline__ void store_out(uint8_t *p, const float (&acc)[N]) {
   }
 }
 
+// One source row of the warp's current item: its byte address (0 = none) and
+// coefficient.  The table lives in shared memory and is re-read (volatile, a
+// broadcast load) on every column vector, so the row addresses do not hold
+// registers: that keeps the kernel at 3-4 resident blocks per SM, i.e. more
+// loads in flight per SM.
+struct SrcEntry {
+  unsigned long long addr;
+  float coef;
+  int aux;  // two-hop: hop-1 row of the source row (-1 = none)
+};
+
+constexpr int kFaninWarps = 8;
+
+__device__ __forceinline__ SrcEntry read_entry(const SrcEntry *e) {
+  uint4 v;
+  asm volatile("ld.volatile.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"((uint32_t)__cvta_generic_to_shared(e)));
+  SrcEntry r;
+  r.addr = ((unsigned long long)v.y << 32) | v.x;
+  r.coef = __uint_as_float(v.z);
+  r.aux = (int)v.w;
+  return r;
+}
+
 template <typename Tin, typename Tout, int KM>
-__global__ void __launch_bounds__(256) fanin_kernel(FaninArgs a, DeviceCtx ctx) {
+__global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
+    fanin_kernel(FaninArgs a, DeviceCtx ctx) {
   constexpr int VE = Elem<Tin>::kPerVec;
+  __shared__ __align__(16) SrcEntry s_tab[kFaninWarps][KM];
   const int lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5;
+  SrcEntry *tab = s_tab[warp];
   int n = a.n_items;
   if (n < 0) n = min(max(*a.n_items_dev, 0), a.cap_items);
   bool bounds = false;
-  for (int item = blockIdx.x * wpb + (threadIdx.x >> 5); item < n; item += gridDim.x * wpb) {
+  for (int item = blockIdx.x * kFaninWarps + warp; item < n; item += gridDim.x * kFaninWarps) {
     int my_r = -1;
     float my_c = 0.0f;
     if (lane < a.k) {
@@ -113,27 +141,31 @@ __global__ void __launch_bounds__(256) fanin_kernel(FaninArgs a, DeviceCtx ctx) 
       if (my_r >= 0) my_c = a.coef ? __ldg(a.coef + my_r) : 1.0f;
     }
     const unsigned vmask = __ballot_sync(kFull, my_r >= 0);
-    int rows[KM];
-    float cf[KM];
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      rows[j] = __shfl_sync(kFull, my_r, j);
-      cf[j] = __shfl_sync(kFull, my_c, j);
+    __syncwarp();  // the previous item's readers are done
+    if (lane < KM) {
+      SrcEntry e;
+      e.addr = my_r >= 0 ? (unsigned long long)(a.y + (size_t)my_r * a.rb_in) : 0ull;
+      e.coef = my_c;
+      e.aux = -1;
+      tab[lane] = e;
     }
+    __syncwarp();
     uint8_t *orow = a.out + (size_t)item * a.rb_out;
     for (int v = lane; v < a.nvec; v += 32) {
       uint4 d[KM];
 #pragma unroll
       for (int j = 0; j < KM; ++j)
-        if (vmask >> j & 1u) d[j] = ld_stream_v4(a.y + (size_t)rows[j] * a.rb_in + (size_t)v * 16);
+        if (vmask >> j & 1u) d[j] = ld_stream_v4((const uint8_t *)read_entry(tab + j).addr + (size_t)v * 16);
       float acc[VE];
 #pragma unroll
       for (int e = 0; e < VE; ++e) acc[e] = 0.0f;
 #pragma unroll
       for (int j = 0; j < KM; ++j)
-        if (vmask >> j & 1u)
+        if (vmask >> j & 1u) {
+          const float c = read_entry(tab + j).coef;
 #pragma unroll
-          for (int e = 0; e < VE; ++e) acc[e] = fmaf(cf[j], Elem<Tin>::get(d[j], e), acc[e]);
+          for (int e = 0; e < VE; ++e) acc[e] = fmaf(c, Elem<Tin>::get(d[j], e), acc[e]);
+        }
       store_out<Tout, VE>(orow + (size_t)v * VE * sizeof(Tout), acc);
     }
   }
@@ -175,12 +207,15 @@ struct TwoHopArgs {
 // summed in ascending group order into the token.  Bit-identical to running
 // the two reverse hops one after the other, without re-reading the partials.
 template <typename Tin, typename Tout, int KM>
-__global__ void __launch_bounds__(256) two_hop_fanin_kernel(TwoHopArgs a, DeviceCtx ctx) {
+__global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
+    two_hop_fanin_kernel(TwoHopArgs a, DeviceCtx ctx) {
   constexpr int VE = Elem<Tin>::kPerVec;
+  __shared__ __align__(16) SrcEntry s_tab[kFaninWarps][KM];
   const int lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5;
+  SrcEntry *tab = s_tab[warp];
   bool bounds = false;
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < a.T; t += gridDim.x * wpb) {
+  for (int t = blockIdx.x * kFaninWarps + warp; t < a.T; t += gridDim.x * kFaninWarps) {
     int my_r = -1, my_s = -1;
     float my_c = 0.0f;
     if (lane < a.k) {
@@ -203,33 +238,37 @@ __global__ void __launch_bounds__(256) two_hop_fanin_kernel(TwoHopArgs a, Device
     // a row closes its group when the next row belongs to another hop-1 row
     const bool closes = my_r >= 0 && (!(vmask >> (lane + 1) & 1u) || lane == 31 || next_s != my_s);
     const unsigned lastmask = __ballot_sync(kFull, closes);
-    int rows[KM], src[KM];
-    float cf[KM];
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      rows[j] = __shfl_sync(kFull, my_r, j);
-      src[j] = __shfl_sync(kFull, my_s, j);
-      cf[j] = __shfl_sync(kFull, my_c, j);
+    __syncwarp();  // the previous token's readers are done
+    if (lane < KM) {
+      SrcEntry e;
+      e.addr = my_r >= 0 ? (unsigned long long)(a.y + (size_t)my_r * a.rb_in) : 0ull;
+      e.coef = my_c;
+      e.aux = my_s;
+      tab[lane] = e;
     }
+    __syncwarp();
     uint8_t *orow = a.out + (size_t)t * a.rb_out;
     for (int v = lane; v < a.nvec; v += 32) {
       uint4 d[KM];
 #pragma unroll
       for (int j = 0; j < KM; ++j)
-        if (vmask >> j & 1u) d[j] = ld_stream_v4(a.y + (size_t)rows[j] * a.rb_in + (size_t)v * 16);
+        if (vmask >> j & 1u) d[j] = ld_stream_v4((const uint8_t *)read_entry(tab + j).addr + (size_t)v * 16);
       float acc_g[VE], acc_o[VE];
 #pragma unroll
       for (int e = 0; e < VE; ++e) acc_g[e] = acc_o[e] = 0.0f;
 #pragma unroll
       for (int j = 0; j < KM; ++j) {
-        if (vmask >> j & 1u)
+        if (vmask >> j & 1u) {
+          const float c = read_entry(tab + j).coef;
 #pragma unroll
-          for (int e = 0; e < VE; ++e) acc_g[e] = fmaf(cf[j], Elem<Tin>::get(d[j], e), acc_g[e]);
+          for (int e = 0; e < VE; ++e) acc_g[e] = fmaf(c, Elem<Tin>::get(d[j], e), acc_g[e]);
+        }
         if (lastmask >> j & 1u) {
 #pragma unroll
           for (int e = 0; e < VE; ++e) acc_g[e] = round_wire<Tin>(acc_g[e]);
-          if (a.hop1 && src[j] >= 0)
-            store_out<Tin, VE>(a.hop1 + (size_t)src[j] * a.rb_in + (size_t)v * 16, acc_g);
+          const int src = read_entry(tab + j).aux;
+          if (a.hop1 && src >= 0)
+            store_out<Tin, VE>(a.hop1 + (size_t)src * a.rb_in + (size_t)v * 16, acc_g);
 #pragma unroll
           for (int e = 0; e < VE; ++e) {
             acc_o[e] += acc_g[e];
@@ -245,11 +284,10 @@ __global__ void __launch_bounds__(256) two_hop_fanin_kernel(TwoHopArgs a, Device
 
 template <typename Tin, typename Tout, int KM>
 cudaError_t launch_two_hop3(const TwoHopArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
-  const int wpb = 8;
-  long blocks = ((long)a.T + wpb - 1) / wpb;
+  long blocks = ((long)a.T + kFaninWarps - 1) / kFaninWarps;
   const long cap = (long)ctx.num_sms * 16;
   if (blocks > cap) blocks = cap;
-  two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, wpb * 32, 0, s>>>(a, ctx);
+  two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
 
@@ -270,12 +308,12 @@ cudaError_t launch_two_hop1(const TwoHopArgs &a, int out_dtype, const DeviceCtx 
 
 template <typename Tin, typename Tout, int KM>
 cudaError_t launch3(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
-  const int wpb = 8;
-  long blocks = (a.n_items >= 0) ? ((long)a.n_items + wpb - 1) / wpb : (long)ctx.num_sms * 8;
+  long blocks = (a.n_items >= 0) ? ((long)a.n_items + kFaninWarps - 1) / kFaninWarps
+                                 : (long)ctx.num_sms * 8;
   const long cap = (long)ctx.num_sms * 16;
   if (blocks > cap) blocks = cap;
   if (blocks <= 0) return cudaSuccess;
-  fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, wpb * 32, 0, s>>>(a, ctx);
+  fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
 
