@@ -7,15 +7,19 @@
 // editorial (lyndhub), section "The core problem".
 //
 // Lane l holds experts l, l+32, l+64, ... of its token (coalesced 128-byte
-// loads).  Softmax max and sum are butterfly reductions, so every lane ends
-// with bit-identical values.  Selection works on an order-preserving u32 key
-// of each logit.  The k-th largest of the 32 lane maxima is a lower bound on
-// the k-th largest key, so only the few elements at or above it can be picked;
-// they are compacted one per lane through shared memory and k rounds of two
-// redux.sync instructions pick the winners: the largest key, and among equal
-// keys the smallest expert id (ties to the lower index).  When more than 32
-// elements tie at the bound, every element is scanned each round instead.
-// The gate weights are computed at the end, one pick per lane.
+// loads).  Selection works on an order-preserving u32 key of each logit; the
+// softmax maximum is the largest key, and the softmax sum a butterfly
+// reduction, so every lane ends with bit-identical values.
+//
+// Selection: the k-th largest of the 32 lane maxima (tau) is a lower bound on
+// the k-th largest key, so only the few elements at or above it can be picked.
+// They are compacted through shared memory in ascending expert order (one
+// ballot per slot), and each candidate counts the candidates that beat it --
+// a larger key, or an equal key at a lower position, i.e. a lower expert id
+// (ties go to the lower index).  That count is its rank; the candidates of rank
+// < k are scattered so lane r holds pick r.  When more than 32 elements tie at
+// the bound, every element is scanned in each of k rounds instead.  The gate
+// weights are computed at the end, one pick per lane.
 #pragma once
 
 #include <math.h>
@@ -28,8 +32,8 @@ namespace route {
 constexpr unsigned kFull = 0xffffffffu;
 
 // Monotone map float -> uint32 (larger float, larger key); -0 and +0 map to
-// the same key so they tie like the floats compare.  Finite values never map
-// to 0, which marks "no candidate".
+// the same key so they tie like the floats compare.  Finite values map into
+// [0x00800000, 0xff800000); -inf, +inf and NaNs land outside that range.
 __device__ __forceinline__ uint32_t order_key(float v) {
   uint32_t u = (v == 0.0f) ? 0u : __float_as_uint(v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -40,67 +44,76 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, d));
-  return v;
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(kFull, v, d);
   return v;
 }
 
-// Per-lane constants of a routing warp.
-template <int EPL>  // experts per lane = ceil(E / 32)
+__device__ __forceinline__ unsigned lanes_below() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Per-lane constants of a routing warp.  FULL: E == 32 * EPL, every slot
+// holds an expert.
+template <int EPL, bool FULL>
 struct Lanes {
   uint32_t valid;  // which of the lane's slots hold an expert
-  int gid[EPL];    // group of each slot (read only when limited)
-  bool limit;
+  bool limit;      // group-limited routing
+  int gsize;       // experts per group
+  uint32_t magic;  // e / gsize == umulhi(e, magic) for e < 2^16, gsize >= 2
 
   __device__ __forceinline__ void init(int lane, int E, int n_groups, int gpt) {
     limit = gpt > 0 && gpt < n_groups;
-    const int gsize = limit ? E / n_groups : E;
+    gsize = limit ? E / n_groups : E;
+    magic = gsize >= 2 ? 0xffffffffu / (uint32_t)gsize + 1u : 0u;
     valid = 0;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E) valid |= 1u << j;
-      gid[j] = limit ? (e < E ? e / gsize : 0) : 0;
-    }
+    for (int j = 0; j < EPL; ++j)
+      if (lane + 32 * j < E) valid |= 1u << j;
+  }
+  __device__ __forceinline__ bool ok(int j) const { return FULL || (valid >> j & 1u); }
+  __device__ __forceinline__ int group(int e) const {
+    return gsize >= 2 ? (int)__umulhi((uint32_t)e, magic) : e;
   }
 };
 
 // Routes the token whose logits start at `row`.  Lanes r < k return pick r in
 // (my_e, my_w); `bad` is set on lanes that saw a non-finite logit.  s_ck and
 // s_ce are this warp's 32-entry shared-memory candidate buffers.
-template <int EPL>
+template <int EPL, bool FULL>
 __device__ __forceinline__ void route_token(const float *row, int E, int k, int n_groups, int gpt,
-                                            int renorm, const Lanes<EPL> &L, uint32_t *s_ck,
+                                            int renorm, const Lanes<EPL, FULL> &L, uint32_t *s_ck,
                                             int *s_ce, int lane, int &my_e, float &my_w,
                                             bool &bad) {
   float v[EPL];
   uint32_t key[EPL];
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    v[j] = (L.valid >> j & 1u) ? __ldcs(row + lane + 32 * j) : 0.0f;
-    bad |= (L.valid >> j & 1u) && !isfinite(v[j]);
-    key[j] = order_key(v[j]);
-  }
-
-  float m = -INFINITY;
+  for (int j = 0; j < EPL; ++j) v[j] = L.ok(j) ? __ldcs(row + lane + 32 * j) : 0.0f;
+  uint32_t kmax = 0, kmin = 0xffffffffu;
 #pragma unroll
-  for (int j = 0; j < EPL; ++j)
-    if (L.valid >> j & 1u) m = fmaxf(m, v[j]);
-  m = warp_max(m);
+  for (int j = 0; j < EPL; ++j) {
+    key[j] = L.ok(j) ? order_key(v[j]) : 0u;
+    if (L.ok(j)) {
+      kmax = max(kmax, key[j]);
+      kmin = min(kmin, key[j]);
+    }
+  }
+  bad |= kmax >= 0xff800000u || kmin < 0x00800000u;
+
+  // softmax maximum and sum over all experts
+  const uint32_t top = __reduce_max_sync(kFull, kmax);
+  const float m = key_value(top);
   float s = 0.0f;
 #pragma unroll
   for (int j = 0; j < EPL; ++j)
-    if (L.valid >> j & 1u) s += expf(v[j] - m);
+    if (L.ok(j)) s += expf(v[j] - m);
   s = warp_sum(s);
 
-  uint32_t avail = L.valid;
+  uint32_t lm = kmax;  // this lane's largest selectable key
+  bool fresh = true;   // lm still equals kmax (then the warp max is `top`)
   if (L.limit) {
     // group score = largest logit in the group; lane g holds group g's key
     uint32_t gkey = 0;
@@ -108,74 +121,73 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
       uint32_t best = 0;
 #pragma unroll
       for (int j = 0; j < EPL; ++j)
-        if ((L.valid >> j & 1u) && L.gid[j] == g) best = max(best, key[j]);
+        if (L.ok(j) && L.group(lane + 32 * j) == g) best = max(best, key[j]);
       best = __reduce_max_sync(kFull, best);
       if (lane == g) gkey = best;
     }
     uint32_t keep = 0;
     for (int r = 0; r < gpt; ++r) {
-      const uint32_t kmax = __reduce_max_sync(kFull, gkey);
-      const int g = (int)__reduce_min_sync(kFull, (gkey == kmax && kmax != 0) ? (unsigned)lane : 32u);
+      const uint32_t gm = __reduce_max_sync(kFull, gkey);
+      const unsigned b = __ballot_sync(kFull, gkey == gm && gm != 0);
+      const int g = b ? __ffs(b) - 1 : 0;
       keep |= 1u << g;
       if (lane == g) gkey = 0;
     }
+    lm = 0;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j)
-      if (!(keep >> L.gid[j] & 1u)) avail &= ~(1u << j);
+    for (int j = 0; j < EPL; ++j) {
+      if (!(keep >> L.group(lane + 32 * j) & 1u)) key[j] = 0;  // 0 = not a candidate
+      lm = max(lm, key[j]);
+    }
+    fresh = false;
   }
-
-#pragma unroll
-  for (int j = 0; j < EPL; ++j)
-    if (!(avail >> j & 1u)) key[j] = 0;  // 0 = not a candidate
 
   // Candidates.  tau = the k-th largest of the 32 lane maxima: k distinct
   // elements reach it, so every top-k element has key >= tau.
-  uint32_t lm = 0;
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) lm = max(lm, key[j]);
   uint32_t tau = 0;
   for (int r = 0; r < k; ++r) {
-    tau = __reduce_max_sync(kFull, lm);
-    const unsigned lw = __reduce_min_sync(kFull, lm == tau ? (unsigned)lane : 32u);
-    if (lane == (int)lw) lm = 0;
+    tau = (r == 0 && fresh) ? top : __reduce_max_sync(kFull, lm);
+    const unsigned b = __ballot_sync(kFull, lm == tau);
+    if (lane == __ffs(b) - 1) lm = 0;
   }
-  int cnt = 0;
+
+  // compaction in ascending expert order: slot j of lane l is expert l + 32 j
+  const unsigned below = lanes_below();
+  unsigned total = 0;
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) cnt += (key[j] >= tau) ? 1 : 0;
-  const unsigned total = __reduce_add_sync(kFull, (unsigned)cnt);
+  for (int j = 0; j < EPL; ++j) {
+    const bool c = L.ok(j) && key[j] >= tau;
+    const unsigned b = __ballot_sync(kFull, c);
+    const unsigned pos = total + __popc(b & below);
+    if (c && pos < 32) {
+      s_ck[pos] = key[j];
+      s_ce[pos] = lane + 32 * j;
+    }
+    total += __popc(b);
+  }
 
   my_e = 0;
   uint32_t my_k = 0;
   if (total <= 32) {
-    // one candidate per lane, through shared memory, then k rounds of
-    // (largest key, then smallest expert id among equal keys)
-    int pos = cnt;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int n = __shfl_up_sync(kFull, pos, d);
-      if (lane >= d) pos += n;
-    }
-    pos -= cnt;
-#pragma unroll
-    for (int j = 0; j < EPL; ++j)
-      if (key[j] >= tau) {
-        s_ck[pos] = key[j];
-        s_ce[pos] = lane + 32 * j;
-        ++pos;
-      }
     __syncwarp();
-    uint32_t ck = lane < (int)total ? s_ck[lane] : 0u;
-    const unsigned ce = lane < (int)total ? (unsigned)s_ce[lane] : 0x7fffffffu;
-    __syncwarp();
-    for (int r = 0; r < k; ++r) {
-      const uint32_t kmax = __reduce_max_sync(kFull, ck);
-      const unsigned ewin = __reduce_min_sync(kFull, ck == kmax ? ce : 0x7fffffffu);
-      if (ce == ewin) ck = 0;
-      if (lane == r) {
-        my_e = (int)ewin;
-        my_k = kmax;
-      }
+    const uint32_t ck = lane < (int)total ? s_ck[lane] : 0u;
+    const int ce = lane < (int)total ? s_ce[lane] : 0;
+    int rank = 0;
+    for (int j = 0; j < (int)total; ++j) {
+      const uint32_t kj = s_ck[j];  // broadcast
+      rank += (kj > ck || (kj == ck && j < lane)) ? 1 : 0;
     }
+    __syncwarp();
+    if (lane < (int)total && rank < k) {
+      s_ck[rank] = ck;
+      s_ce[rank] = ce;
+    }
+    __syncwarp();
+    if (lane < k) {
+      my_k = s_ck[lane];
+      my_e = s_ce[lane];
+    }
+    __syncwarp();
   } else {
     // many ties at tau: scan every element each round
     for (int r = 0; r < k; ++r) {
@@ -187,8 +199,8 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
           bk = key[j];
           be = lane + 32 * j;
         }
-      const uint32_t kmax = __reduce_max_sync(kFull, bk);
-      const int ewin = (int)__reduce_min_sync(kFull, (bk == kmax) ? (unsigned)be : 0x7fffffffu);
+      const uint32_t kmx = __reduce_max_sync(kFull, bk);
+      const int ewin = (int)__reduce_min_sync(kFull, (bk == kmx) ? (unsigned)be : 0x7fffffffu);
       if (lane == (ewin & 31)) {
 #pragma unroll
         for (int j = 0; j < EPL; ++j)
@@ -196,7 +208,7 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
       }
       if (lane == r) {
         my_e = ewin;
-        my_k = kmax;
+        my_k = kmx;
       }
     }
   }

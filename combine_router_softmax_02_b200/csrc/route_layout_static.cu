@@ -27,7 +27,7 @@ struct RouteArgs {
   int *rank_active;  // [R] activated experts per rank, or null
 };
 
-template <int EPL>
+template <int EPL, bool FULL>
 __global__ void __launch_bounds__(256) route_count_kernel(RouteArgs ra, LayoutArgs a, DeviceCtx ctx) {
   __shared__ uint32_t s_ck[8][32];
   __shared__ int s_ce[8][32];
@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(256) route_count_kernel(RouteArgs ra, LayoutAr
     a.state[i] = 0ull;
   __syncthreads();
 
-  route::Lanes<EPL> L;
+  route::Lanes<EPL, FULL> L;
   L.init(lane, a.E, ra.n_groups, ra.gpt);
   // contiguous tokens per block, so each block touches few source ranks
   const int per = ((a.T + gridDim.x - 1) / gridDim.x + 7) & ~7;
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) route_count_kernel(RouteArgs ra, LayoutAr
   for (int t = t0 + warp; t < t1; t += 8) {
     int e;
     float w;
-    route::route_token<EPL>(ra.logits + (size_t)t * a.E, a.E, a.k, ra.n_groups, ra.gpt, ra.renorm, L,
+    route::route_token<EPL, FULL>(ra.logits + (size_t)t * a.E, a.E, a.k, ra.n_groups, ra.gpt, ra.renorm, L,
                             s_ck[warp], s_ce[warp], lane, e, w, bad);
     int r = -1;
     if (lane < a.k) {
@@ -122,7 +122,10 @@ cudaError_t launch_epl(const RouteArgs &ra, const LayoutArgs &a, const DeviceCtx
   long blocks = ((long)a.T + 63) / 64;  // >= 64 tokens per block
   const long cap = (long)ctx.num_sms * 4;
   if (blocks > cap) blocks = cap;
-  route_count_kernel<EPL><<<(unsigned)blocks, 256, 0, s>>>(ra, a, ctx);
+  if (a.E == 32 * EPL)
+    route_count_kernel<EPL, true><<<(unsigned)blocks, 256, 0, s>>>(ra, a, ctx);
+  else
+    route_count_kernel<EPL, false><<<(unsigned)blocks, 256, 0, s>>>(ra, a, ctx);
   return count_launch(cudaGetLastError());
 }
 

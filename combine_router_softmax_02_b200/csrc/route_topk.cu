@@ -4,7 +4,7 @@
 namespace moe {
 namespace {
 
-template <int EPL>
+template <int EPL, bool FULL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
                                                          int E, int k, int n_groups, int gpt,
                                                          int renorm, int *__restrict__ idx_out,
@@ -14,13 +14,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int wpb = blockDim.x >> 5;
-  route::Lanes<EPL> L;
+  route::Lanes<EPL, FULL> L;
   L.init(lane, E, n_groups, gpt);
   for (int t = blockIdx.x * wpb + warp; t < T; t += gridDim.x * wpb) {
     int my_e;
     float my_w;
     bool bad = false;
-    route::route_token<EPL>(logits + (size_t)t * E, E, k, n_groups, gpt, renorm, L, s_ck[warp],
+    route::route_token<EPL, FULL>(logits + (size_t)t * E, E, k, n_groups, gpt, renorm, L, s_ck[warp],
                             s_ce[warp], lane, my_e, my_w, bad);
     if (__any_sync(route::kFull, bad) && lane == 0) set_status(ctx.status, MOE_ERR_BAD_INPUT);
     if (lane < k) {
@@ -37,8 +37,12 @@ cudaError_t launch_epl(const float *logits, int T, int E, int k, int n_groups, i
   long blocks = (T + wpb - 1) / wpb;
   const long cap = (long)ctx.num_sms * 16;
   if (blocks > cap) blocks = cap;
-  route_topk_kernel<EPL><<<(unsigned)blocks, wpb * 32, 0, s>>>(logits, T, E, k, n_groups, gpt,
-                                                               renorm, idx, w, ctx);
+  if (E == 32 * EPL)
+    route_topk_kernel<EPL, true><<<(unsigned)blocks, wpb * 32, 0, s>>>(logits, T, E, k, n_groups,
+                                                                      gpt, renorm, idx, w, ctx);
+  else
+    route_topk_kernel<EPL, false><<<(unsigned)blocks, wpb * 32, 0, s>>>(logits, T, E, k, n_groups,
+                                                                       gpt, renorm, idx, w, ctx);
   return count_launch(cudaGetLastError());
 }
 
