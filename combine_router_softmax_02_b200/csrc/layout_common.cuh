@@ -1,6 +1,19 @@
-// Pieces of the layout shared by the layout kernels and the fused
-// static-placement kernel: arguments, warp helpers, and the final scan of the
-// per-bin totals into segment offsets (see build_layout.cu).
+// Pieces of the layout shared by the layout kernel (build_layout.cu) and the
+// fused static-placement kernel (route_layout_static.cu): arguments, the
+// shared-memory plan, per-token pick loading, warp bin ballots, the grid
+// barrier, and the second phase that turns bin counts into rows.
+//
+// One launch, two phases.  Every block owns a contiguous chunk of tokens.
+// Phase 1 counts the rows of every bin ("bins" are ranks for DEDUP, ranks then
+// groups for TWO_HOP, experts for PER_PICK) over the block's chunk and stores
+// the counts in its row of the workspace.  After a grid barrier every block
+// reads all blocks' counts: their sum per bin gives the segment offsets, the
+// sum over earlier blocks its own base in every bin.  Phase 2 then walks the
+// chunk again in tiles of 256 tokens; within a tile a warp's ballot of a bin
+// gives both the bin's count in the warp and each lane's position (token
+// order), and one thread per bin scans the warps.  The grid is sized so that
+// every block is resident at once (cooperative launch) and the barrier wait is
+// bounded.
 #pragma once
 
 #include "moe_internal.cuh"
@@ -8,42 +21,99 @@
 namespace moe {
 namespace layout {
 
-constexpr int kTile = 256;  // tokens per tile, one per thread
+constexpr int kTile = 256;  // threads per block, tokens per phase-2 tile
 constexpr int kWarps = kTile / 32;
 constexpr int kMaxBins = kMaxE;  // >= max(E, R + G)
-constexpr int kSendSmem = kMaxR * kMaxR;
+constexpr int kMaxBlocks = 512;  // grid cap (rows of the count table)
+constexpr int kBlocksPerSm = 2;  // layout grid: blocks per SM (when resident)
+constexpr int kHeaderInts = 16;  // barrier words at the start of the workspace
 constexpr unsigned kFull = 0xffffffffu;
-constexpr unsigned long long kFlagAgg = 1ull << 32;
-constexpr unsigned long long kFlagInc = 2ull << 32;
 
 struct LayoutArgs {
   const int *idx;
   const float *w;
   const int *expert_rank;
-  int T, tpr, k, E, R, rpg, G, mode, NB, num_tiles;
-  int *counters;  // [0] place-kernel ticket, [1] count-kernel blocks done
-  int *totals;    // [NB]
-  int *seg_off;   // [NB]
-  unsigned long long *state;  // [num_tiles][NB]: flag << 32 | count
+  int T, tpr, k, E, R, rpg, G, mode, NB, NBp;
+  int nblk;        // blocks of the launch
+  int chunk;       // tokens per block, a multiple of 32
+  unsigned *bar;   // [0] barrier arrivals, [1] blocks done
+  int *agg;        // [nblk][NBp] per-block bin counts
   moe_layout L;
 };
 
-__device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
-  const unsigned lo = __reduce_or_sync(kFull, (unsigned)m);
-  const unsigned hi = __reduce_or_sync(kFull, (unsigned)(m >> 32));
-  return ((unsigned long long)hi << 32) | lo;
+// Shared memory of one block, in ints.
+struct SmemPlan {
+  int er, cnt, base, w, woff, ptot, ppre, seg, send, hist, total;
+};
+
+__host__ __device__ inline SmemPlan smem_plan(int E, int NBp, int R, bool fused) {
+  SmemPlan s;
+  int o = 0;
+  s.er = o;   o += (E + 3) & ~3;
+  s.cnt = o;  o += NBp;           // block counts, then per-bin totals
+  s.base = o; o += NBp;           // running row base of every bin
+  s.w = o;    o += kWarps * NBp;  // per-warp ballots (mask bins) or counts (experts)
+  s.woff = o; o += kWarps * NBp;  // per-warp row offsets (mask bins)
+  s.ptot = o; o += 1024;          // partial sums of the count table
+  s.ppre = o; o += 1024;
+  s.seg = o;  o += NBp + 2 * kMaxR + 4;  // segment offsets, rank totals and bases
+  s.send = o; o += R * R;         // the block's send-count matrix
+  s.hist = o; o += fused ? ((E + 3) & ~3) : 0;
+  s.total = o;
+  return s;
 }
 
-// Bins given as 64-bit masks (ranks, or groups): for every bin present in the
-// warp, f(bin, has, ball) runs on all lanes with the warp's ballot of the bin.
-template <class F>
-__device__ __forceinline__ void warp_mask_bins(unsigned long long mask, F &&f) {
-  unsigned long long wm = warp_or64(mask);
-  while (wm) {
-    const int b = __ffsll((long long)wm) - 1;
-    wm &= wm - 1;
-    const bool has = (mask >> b) & 1ull;
-    f(b, has, __ballot_sync(kFull, has));
+// ---------------------------------------------------------------- tokens ----
+// One token's picks as seen by one thread.
+template <int KM>
+struct TokenPicks {
+  int e[KM];
+  int r[KM];
+  float w[KM];
+  uint32_t present;          // picks with a valid expert and rank
+  unsigned long long dmask;  // ranks of the token
+  unsigned long long gmask;  // groups of the token (TWO_HOP)
+};
+
+template <int KM>
+__device__ __forceinline__ void load_picks(const LayoutArgs &a, const int *s_er, int t, bool live,
+                                           bool want_w, TokenPicks<KM> &p, bool &bad) {
+  p.present = 0;
+  p.dmask = 0;
+  p.gmask = 0;
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    p.e[j] = 0;
+    p.r[j] = 0;
+    p.w[j] = 0.0f;
+    if (j < a.k && live) {
+      const int e = a.idx[(size_t)t * a.k + j];
+      if ((unsigned)e < (unsigned)a.E) {
+        const int r = s_er[e];
+        if ((unsigned)r < (unsigned)a.R) {
+          p.e[j] = e;
+          p.r[j] = r;
+          p.present |= 1u << j;
+          p.dmask |= 1ull << r;
+          p.gmask |= 1ull << (r / a.rpg);
+          if (want_w) p.w[j] = a.w[(size_t)t * a.k + j];
+        } else {
+          bad = true;
+        }
+      } else {
+        bad = true;
+      }
+    }
+  }
+  if (a.mode == MOE_LAYOUT_PER_PICK) {  // the row order needs distinct experts per token
+#pragma unroll
+    for (int i = 0; i < KM; ++i)
+#pragma unroll
+      for (int j = i + 1; j < KM; ++j)
+        if ((p.present >> i & 1u) && (p.present >> j & 1u) && p.e[i] == p.e[j]) {
+          bad = true;
+          p.present &= ~(1u << j);
+        }
   }
 }
 
@@ -53,65 +123,466 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
+__device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
+  const unsigned lo = __reduce_or_sync(kFull, (unsigned)m);
+  const unsigned hi = __reduce_or_sync(kFull, (unsigned)(m >> 32));
+  return ((unsigned long long)hi << 32) | lo;
+}
+
 __device__ __forceinline__ unsigned long long group_bits(int g, int rpg) {
   const unsigned long long ones = (rpg >= 64) ? ~0ull : ((1ull << rpg) - 1ull);
   return (rpg >= 64) ? ones : (ones << (g * rpg));
 }
 
-// ------------------------------------------------------------- finalize ----
-// Runs in the last count block, all threads: the totals are loaded into
-// shared memory in parallel (tot), then thread 0 scans them into segment
-// offsets and the host-visible offsets.
-__device__ __forceinline__ void finalize(const LayoutArgs &a, const int *s_er, int *tot, DeviceCtx ctx) {
-  for (int i = threadIdx.x; i < a.NB; i += blockDim.x) tot[i] = __ldcg(a.totals + i);
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  const moe_layout &L = a.L;
-  if (a.mode == MOE_LAYOUT_PER_PICK) {
-    int base[kMaxR + 1];
-    for (int r = 0; r <= a.R; ++r) base[r] = 0;
-    for (int e = 0; e < a.E; ++e) {
-      const int r = s_er[e];
-      if ((unsigned)r < (unsigned)a.R) base[r + 1] += tot[e];
-    }
-    for (int r = 0; r < a.R; ++r) base[r + 1] += base[r];
-    for (int r = 0; r <= a.R; ++r) L.rank_offsets[r] = base[r];
-    const int n = base[a.R];
-    for (int e = 0; e < a.E; ++e) {
-      const int r = s_er[e];
-      if ((unsigned)r < (unsigned)a.R) {
-        a.seg_off[e] = base[r];
-        base[r] += tot[e];
-      } else {
-        a.seg_off[e] = 0;
-      }
-    }
-    *L.num_rows = n;
-    if (n > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
-    return;
+// The warp's ballots of bins [0, n) (n <= 64) of a 64-bit mask per lane:
+// lane i gets the ballots of bins i (b0) and i + 32 (b1).
+__device__ __forceinline__ void warp_bin_ballots(unsigned long long m, int n, int lane,
+                                                 unsigned &b0, unsigned &b1) {
+  b0 = 0;
+  b1 = 0;
+  const unsigned lo = (unsigned)m, hi = (unsigned)(m >> 32);
+  const int n0 = n < 32 ? n : 32;
+#pragma unroll 8
+  for (int i = 0; i < n0; ++i) {
+    const unsigned bal = __ballot_sync(kFull, (lo >> i) & 1u);
+    if (lane == i) b0 = bal;
   }
-  int run = 0;
-  for (int r = 0; r < a.R; ++r) {
-    a.seg_off[r] = run;
-    L.rank_offsets[r] = run;
-    run += tot[r];
-  }
-  L.rank_offsets[a.R] = run;
-  *L.num_rows = run;
-  if (run > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
-  if (a.mode == MOE_LAYOUT_TWO_HOP) {
-    int run1 = 0;
-    for (int g = 0; g < a.G; ++g) {
-      a.seg_off[a.R + g] = run1;
-      L.group_offsets[g] = run1;
-      run1 += tot[a.R + g];
-    }
-    L.group_offsets[a.G] = run1;
-    *L.num_rows_hop1 = run1;
-    if (run1 > L.capacity_hop1) set_status(ctx.status, MOE_ERR_CAPACITY);
+#pragma unroll 8
+  for (int i = 32; i < n; ++i) {
+    const unsigned bal = __ballot_sync(kFull, (hi >> (i - 32)) & 1u);
+    if (lane == i - 32) b1 = bal;
   }
 }
 
+// ------------------------------------------------------------- experts ----
+// Merge the lanes' distinct (rank << 10 | expert) keys in ascending order.  For
+// every key present in the warp, f(key, has, ball, c, matched) runs on all
+// lanes: `has` says whether this lane's token has the key, `ball` which lanes
+// do, `c` how many distinct keys this lane had before, `matched` its picks
+// with the key.
+template <int KM, class F>
+__device__ __forceinline__ void warp_merge(const TokenPicks<KM> &p, F &&f) {
+  uint32_t key[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) key[j] = ((uint32_t)p.r[j] << 10) | (uint32_t)p.e[j];
+  uint32_t rem = p.present;
+  int c = 0;
+  while (true) {
+    uint32_t mine = 0xffffffffu;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (rem >> j & 1u) mine = min(mine, key[j]);
+    const uint32_t b = __reduce_min_sync(kFull, mine);
+    if (b == 0xffffffffu) break;
+    const bool has = (mine == b);
+    const unsigned ball = __ballot_sync(kFull, has);
+    uint32_t matched = 0;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if ((rem >> j & 1u) && key[j] == b) matched |= 1u << j;
+    f(b, has, ball, c, matched);
+    if (has) {
+      rem &= ~matched;
+      ++c;
+    }
+  }
+}
+
+// ------------------------------------------------------------- phase 1 ----
+// Adds one tile's bin counts of this warp into lane-held totals: c[0], c[1]
+// for ranks lane and lane + 32, c[2], c[3] for groups lane and lane + 32
+// (mask modes); experts go straight to the block counts (PER_PICK).
+template <int KM>
+__device__ __forceinline__ void count_tile(const LayoutArgs &a, const TokenPicks<KM> &p, int lane,
+                                           int *s_cnt, int (&c)[4]) {
+  if (a.mode == MOE_LAYOUT_PER_PICK) {
+    warp_merge<KM>(p, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
+      if (lane == 0) atomicAdd(&s_cnt[b & 1023u], __popc(ball));
+    });
+    return;
+  }
+  unsigned b0, b1;
+  warp_bin_ballots(p.dmask, a.R, lane, b0, b1);
+  c[0] += __popc(b0);
+  c[1] += __popc(b1);
+  if (a.mode == MOE_LAYOUT_TWO_HOP) {
+    warp_bin_ballots(p.gmask, a.G, lane, b0, b1);
+    c[2] += __popc(b0);
+    c[3] += __popc(b1);
+  }
+}
+
+// Moves the lane-held mask-bin totals into the block counts.
+__device__ __forceinline__ void flush_counts(const LayoutArgs &a, int lane, int *s_cnt,
+                                             const int (&c)[4]) {
+  if (a.mode == MOE_LAYOUT_PER_PICK) return;
+  if (lane < a.R && c[0]) atomicAdd(&s_cnt[lane], c[0]);
+  if (lane + 32 < a.R && c[1]) atomicAdd(&s_cnt[lane + 32], c[1]);
+  if (a.mode == MOE_LAYOUT_TWO_HOP) {
+    if (lane < a.G && c[2]) atomicAdd(&s_cnt[a.R + lane], c[2]);
+    if (lane + 32 < a.G && c[3]) atomicAdd(&s_cnt[a.R + lane + 32], c[3]);
+  }
+}
+
+// ------------------------------------------------------------- barrier ----
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier over the launch's blocks (all resident: cooperative
+// launch).  Returns false on every thread of the block when the wait ran out
+// (MOE_ERR_TIMEOUT is set) or the block is the test hook's silent block, which
+// never arrives.
+__device__ __forceinline__ bool grid_barrier(const LayoutArgs &a, const DeviceCtx &ctx, int *s_flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    if ((int)blockIdx.x == ctx.silent_tile) {
+      ok = 0;
+    } else {
+      red_release_add(a.bar, 1u);
+      if (ld_acquire_u32(a.bar) < (unsigned)a.nblk) {
+        const uint64_t t0 = global_ns();
+        while (ld_acquire_u32(a.bar) < (unsigned)a.nblk) {
+          __nanosleep(32);
+          if (global_ns() - t0 > ctx.wait_limit_ns || ld_volatile_i32(ctx.status) == MOE_ERR_TIMEOUT) {
+            set_status(ctx.status, MOE_ERR_TIMEOUT);
+            ok = 0;
+            break;
+          }
+        }
+      }
+    }
+    *s_flag = ok;
+  }
+  __syncthreads();
+  return *s_flag != 0;
+}
+
+// ------------------------------------------------------------- phase 2 ----
+// Per-bin totals (into s_cnt) and this block's base (into s_base) from the
+// count table, then the segment offsets; block 0 writes the layout's offsets.
+__device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const SmemPlan &P, int *sm,
+                                                  DeviceCtx ctx) {
+  const int tid = threadIdx.x;
+  const int V = a.NBp / 4;                      // 16-byte vectors per table row
+  const int Q = V >= kTile ? 1 : kTile / V;     // row groups
+  int *s_cnt = sm + P.cnt, *s_base = sm + P.base, *s_ptot = sm + P.ptot, *s_ppre = sm + P.ppre;
+  const int blk = blockIdx.x;
+  for (int x = tid; x < Q * V; x += kTile) {
+    const int q = x / V, v = x % V;
+    int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
+#pragma unroll 4
+    for (int g = q; g < a.nblk; g += Q) {
+      const int4 c = __ldcg(reinterpret_cast<const int4 *>(a.agg + (size_t)g * a.NBp) + v);
+      tot.x += c.x; tot.y += c.y; tot.z += c.z; tot.w += c.w;
+      if (g < blk) {
+        pre.x += c.x; pre.y += c.y; pre.z += c.z; pre.w += c.w;
+      }
+    }
+    reinterpret_cast<int4 *>(s_ptot + q * a.NBp)[v] = tot;
+    reinterpret_cast<int4 *>(s_ppre + q * a.NBp)[v] = pre;
+  }
+  __syncthreads();
+  for (int b = tid; b < a.NB; b += kTile) {
+    int tot = 0, pre = 0;
+    for (int q = 0; q < Q; ++q) {
+      tot += s_ptot[q * a.NBp + b];
+      pre += s_ppre[q * a.NBp + b];
+    }
+    s_cnt[b] = tot;
+    s_base[b] = pre;
+  }
+  __syncthreads();
+
+  // segment offsets
+  int *s_seg = sm + P.seg;
+  int *s_rtot = s_seg + a.NBp;    // PER_PICK: rows per rank
+  int *s_rbase = s_rtot + kMaxR;  // PER_PICK: first row of each rank
+  const int *s_er = sm + P.er;
+  const moe_layout &L = a.L;
+  const int lane = tid & 31;
+  if (a.mode == MOE_LAYOUT_PER_PICK) {
+    if (tid < a.R) {  // each rank walks its experts in ascending order
+      int run = 0;
+      for (int e = 0; e < a.E; ++e)
+        if (s_er[e] == tid) {
+          s_seg[e] = run;
+          run += s_cnt[e];
+        }
+      s_rtot[tid] = run;
+    }
+    __syncthreads();
+    if (tid < 32) {  // exclusive scan of the rank totals (R <= 64)
+      const int v0 = lane < a.R ? s_rtot[lane] : 0, v1 = lane + 32 < a.R ? s_rtot[lane + 32] : 0;
+      int i0 = v0, i1 = v1;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int n0 = __shfl_up_sync(kFull, i0, d), n1 = __shfl_up_sync(kFull, i1, d);
+        if (lane >= d) {
+          i0 += n0;
+          i1 += n1;
+        }
+      }
+      const int tot0 = __shfl_sync(kFull, i0, 31);
+      const int tot1 = __shfl_sync(kFull, i1, 31);  // every lane takes part
+      if (lane < a.R) s_rbase[lane] = i0 - v0;
+      if (lane + 32 < a.R) s_rbase[lane + 32] = tot0 + i1 - v1;
+      if (lane == 0) s_rbase[kMaxR] = tot0 + tot1;
+    }
+    __syncthreads();
+    for (int e = tid; e < a.E; e += kTile) {
+      const int r = s_er[e];
+      s_seg[e] = ((unsigned)r < (unsigned)a.R) ? s_seg[e] + s_rbase[r] : 0;
+    }
+    if (blk == 0) {
+      for (int r = tid; r <= a.R; r += kTile) L.rank_offsets[r] = r < a.R ? s_rbase[r] : s_rbase[kMaxR];
+      if (tid == 0) {
+        const int n = s_rbase[kMaxR];
+        *L.num_rows = n;
+        if (n > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
+      }
+    }
+  } else if (tid < 32) {
+    // exclusive scans of the rank totals and of the group totals (<= 64 each)
+    for (int part = 0; part < (a.mode == MOE_LAYOUT_TWO_HOP ? 2 : 1); ++part) {
+      const int n = part ? a.G : a.R, off = part ? a.R : 0;
+      const int v0 = lane < n ? s_cnt[off + lane] : 0, v1 = lane + 32 < n ? s_cnt[off + lane + 32] : 0;
+      int i0 = v0, i1 = v1;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int n0 = __shfl_up_sync(kFull, i0, d), n1 = __shfl_up_sync(kFull, i1, d);
+        if (lane >= d) {
+          i0 += n0;
+          i1 += n1;
+        }
+      }
+      const int tot0 = __shfl_sync(kFull, i0, 31);
+      const int total = tot0 + __shfl_sync(kFull, i1, 31);
+      if (lane < n) s_seg[off + lane] = i0 - v0;
+      if (lane + 32 < n) s_seg[off + lane + 32] = tot0 + i1 - v1;
+      if (blk == 0) {
+        int *offs = part ? L.group_offsets : L.rank_offsets;
+        if (lane < n) offs[lane] = i0 - v0;
+        if (lane + 32 < n) offs[lane + 32] = tot0 + i1 - v1;
+        if (lane == 0) {
+          offs[n] = total;
+          if (part == 0) {
+            *L.num_rows = total;
+            if (total > L.capacity) set_status(ctx.status, MOE_ERR_CAPACITY);
+          } else {
+            *L.num_rows_hop1 = total;
+            if (total > L.capacity_hop1) set_status(ctx.status, MOE_ERR_CAPACITY);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int b = tid; b < a.NB; b += kTile) s_base[b] += s_seg[b];
+  __syncthreads();
+}
+
+// Rows of one tile of mask-bin tokens (DEDUP, TWO_HOP).  Every thread of the
+// block calls it; `t` is the thread's token, `live` whether it has one.
+template <int KM>
+__device__ __forceinline__ void rows_mask_tile(const LayoutArgs &a, const SmemPlan &P, int *sm,
+                                               const TokenPicks<KM> &p, int t, bool live, bool &over) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int *s_w = sm + P.w + warp * a.NBp;
+  const int *s_woff = sm + P.woff + warp * a.NBp;
+  unsigned b0, b1, g0 = 0, g1 = 0;
+  warp_bin_ballots(p.dmask, a.R, lane, b0, b1);
+  if (lane < a.R) s_w[lane] = b0;
+  if (lane + 32 < a.R) s_w[lane + 32] = b1;
+  if (a.mode == MOE_LAYOUT_TWO_HOP) {
+    warp_bin_ballots(p.gmask, a.G, lane, g0, g1);
+    if (lane < a.G) s_w[a.R + lane] = g0;
+    if (lane + 32 < a.G) s_w[a.R + lane + 32] = g1;
+  }
+  // send counts: source rank of the token -> its ranks
+  int *s_send = sm + P.send;
+  const int src = live ? t / a.tpr : 0;
+  const int src0 = __shfl_sync(kFull, src, 0);
+  if (__all_sync(kFull, !live || src == src0)) {
+    if (b0) atomicAdd(&s_send[src0 * a.R + lane], __popc(b0));
+    if (b1) atomicAdd(&s_send[src0 * a.R + lane + 32], __popc(b1));
+  } else {
+    for (unsigned long long m = p.dmask; m; m &= m - 1)
+      atomicAdd(&s_send[src * a.R + __ffsll((long long)m) - 1], 1);
+  }
+  __syncthreads();
+  int *s_base = sm + P.base;
+  for (int b = tid; b < a.NB; b += kTile) {
+    int run = s_base[b];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      sm[P.woff + w * a.NBp + b] = run;
+      run += __popc((unsigned)sm[P.w + w * a.NBp + b]);
+    }
+    s_base[b] = run;
+  }
+  __syncthreads();
+
+  const moe_layout &L = a.L;
+  const unsigned lt = lanemask_lt();
+  const size_t tk = (size_t)t * a.k;
+  auto row_of = [&](int bin) { return s_woff[bin] + __popc((unsigned)s_w[bin] & lt); };
+  if (a.mode == MOE_LAYOUT_TWO_HOP) {
+    int cg = 0;
+    for (unsigned long long m = p.gmask; m; m &= m - 1, ++cg) {
+      const int g = __ffsll((long long)m) - 1;
+      const int row1 = row_of(a.R + g);
+      if (row1 < L.capacity_hop1) {
+        L.hop1_row_token[row1] = t;
+        L.token_groups[tk + cg] = row1;
+        const int nchild = __popcll(p.dmask & group_bits(g, a.rpg));
+        for (int ci = nchild; ci < a.k; ++ci) L.hop1_children[(size_t)row1 * a.k + ci] = -1;
+      } else {
+        L.token_groups[tk + cg] = -1;
+        over = true;
+      }
+    }
+    if (live)
+      for (int c = cg; c < a.k; ++c) L.token_groups[tk + c] = -1;
+  }
+  int c = 0;
+  for (unsigned long long m = p.dmask; m; m &= m - 1, ++c) {
+    const int r = __ffsll((long long)m) - 1;
+    const int row = row_of(r);
+    float coef = 0.0f;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if ((p.present >> j & 1u) && p.r[j] == r) coef += p.w[j];
+    const bool fits = row < L.capacity;
+    if (fits) {
+      L.row_token[row] = t;
+      L.row_coef[row] = coef;
+      L.token_rows[tk + c] = row;
+    } else {
+      L.token_rows[tk + c] = -1;
+      over = true;
+    }
+    if (a.mode == MOE_LAYOUT_TWO_HOP) {
+      const int g = r / a.rpg;
+      int row1 = row_of(a.R + g);
+      if (row1 >= L.capacity_hop1) row1 = -1;
+      const int ci = __popcll(p.dmask & group_bits(g, a.rpg) & ((1ull << r) - 1ull));
+      if (fits) L.hop2_src_row[row] = row1;
+      if (row1 >= 0) L.hop1_children[(size_t)row1 * a.k + ci] = fits ? row : -1;
+    }
+  }
+  if (live)
+    for (int cc = c; cc < a.k; ++cc) L.token_rows[tk + cc] = -1;
+  __syncthreads();  // s_w and s_woff are reused by the next tile
+}
+
+// Rows of one tile of PER_PICK tokens: rows (rank, expert, token).
+template <int KM>
+__device__ __forceinline__ void rows_pick_tile(const LayoutArgs &a, const SmemPlan &P, int *sm,
+                                               const TokenPicks<KM> &p, int t, bool live, bool &over) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kWarps * a.NBp; i += kTile) sm[P.w + i] = 0;
+  __syncthreads();
+  int *s_w = sm + P.w + warp * a.NBp;
+  int *s_send = sm + P.send;
+  const int src = live ? t / a.tpr : 0;
+  const int src0 = __shfl_sync(kFull, src, 0);
+  const bool uniform = __all_sync(kFull, !live || src == src0);
+  warp_merge<KM>(p, [&](uint32_t b, bool has, unsigned ball, int, uint32_t) {
+    if (lane == 0) s_w[b & 1023u] = __popc(ball);
+    if (!has) return;
+    const unsigned peers = uniform ? ball : __match_any_sync(ball, src);
+    if (lane == __ffs(peers) - 1) atomicAdd(&s_send[src * a.R + (int)(b >> 10)], __popc(peers));
+  });
+  __syncthreads();
+  int *s_base = sm + P.base;
+  for (int b = tid; b < a.NB; b += kTile) {
+    int run = s_base[b];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = sm[P.w + w * a.NBp + b];
+      sm[P.w + w * a.NBp + b] = run;
+      run += c;
+    }
+    s_base[b] = run;
+  }
+  __syncthreads();
+  const moe_layout &L = a.L;
+  const unsigned lt = lanemask_lt();
+  const size_t tk = (size_t)t * a.k;
+  int cnt = 0;
+  warp_merge<KM>(p, [&](uint32_t b, bool has, unsigned ball, int c, uint32_t matched) {
+    if (!has) return;
+    const int row = s_w[b & 1023u] + __popc(ball & lt);
+    float coef = 0.0f;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (matched >> j & 1u) coef += p.w[j];
+    if (row < L.capacity) {
+      L.row_token[row] = t;
+      L.row_coef[row] = coef;
+      L.token_rows[tk + c] = row;
+    } else {
+      L.token_rows[tk + c] = -1;
+      over = true;
+    }
+    cnt = c + 1;
+  });
+  if (live)
+    for (int c = cnt; c < a.k; ++c) L.token_rows[tk + c] = -1;
+  __syncthreads();
+}
+
+// Phase 2 of the block's chunk [t0, t1) once the barrier has passed.
+template <int KM>
+__device__ __forceinline__ void phase2(const LayoutArgs &a, const SmemPlan &P, int *sm, int t0,
+                                       int t1, DeviceCtx ctx) {
+  bases_from_counts(a, P, sm, ctx);
+  bool over = false, bad = false;
+  for (int base = t0; base < t1; base += kTile) {
+    const int t = base + (int)threadIdx.x;
+    const bool live = t < t1;
+    TokenPicks<KM> p;
+    load_picks<KM>(a, sm + P.er, t, live, true, p, bad);
+    if (a.mode == MOE_LAYOUT_PER_PICK)
+      rows_pick_tile<KM>(a, P, sm, p, t, live, over);
+    else
+      rows_mask_tile<KM>(a, P, sm, p, t, live, over);
+  }
+  if (over) set_status(ctx.status, MOE_ERR_CAPACITY);
+  // the block's send counts (send_counts was cleared before the barrier)
+  const int *s_send = sm + P.send;
+  for (int i = threadIdx.x; i < a.R * a.R; i += kTile)
+    if (s_send[i]) atomicAdd(&a.L.send_counts[i], s_send[i]);
+}
+
+// Phase-1 epilogue: the block's counts into its table row; block 0 clears the
+// send-count matrix (every block adds into it after the barrier).
+__device__ __forceinline__ void publish_counts(const LayoutArgs &a, const SmemPlan &P, int *sm) {
+  __syncthreads();
+  for (int b = threadIdx.x; b < a.NBp; b += kTile)
+    a.agg[(size_t)blockIdx.x * a.NBp + b] = b < a.NB ? sm[P.cnt + b] : 0;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < a.R * a.R; i += kTile) a.L.send_counts[i] = 0;
+}
+
+// Clears the block's shared counters and loads the expert -> rank map.
+__device__ __forceinline__ void smem_init(const LayoutArgs &a, const SmemPlan &P, int *sm) {
+  for (int i = threadIdx.x; i < a.E; i += kTile) sm[P.er + i] = a.expert_rank[i];
+  for (int i = threadIdx.x; i < a.NBp; i += kTile) sm[P.cnt + i] = 0;
+  for (int i = threadIdx.x; i < a.R * a.R; i += kTile) sm[P.send + i] = 0;
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- host ----
 inline int num_bins(int E, int R, int rpg, int mode) {
   if (mode == MOE_LAYOUT_PER_PICK) return E;
   if (mode == MOE_LAYOUT_TWO_HOP) return R + R / rpg;
@@ -120,17 +591,24 @@ inline int num_bins(int E, int R, int rpg, int mode) {
 
 inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
 
+// Blocks and chunk of a launch: at most `max_blocks` blocks, chunks of a
+// multiple of 32 tokens.
+inline void split_tokens(int T, int max_blocks, int &nblk, int &chunk) {
+  if (max_blocks < 1) max_blocks = 1;
+  if (max_blocks > kMaxBlocks) max_blocks = kMaxBlocks;
+  chunk = (int)(((long)T + max_blocks - 1) / max_blocks);
+  chunk = (chunk + 31) & ~31;
+  nblk = (int)(((long)T + chunk - 1) / chunk);
+}
+
 // Arguments of one layout over the caller's buffers and workspace.
 LayoutArgs make_layout_args(const int *idx, const float *w, const int *expert_rank, int T,
                             int tokens_per_rank, int k, int E, int R, int rpg, int mode,
                             const moe_layout &L, void *ws);
-// Clears the counters, totals and the send-count matrix (stream-ordered).
-cudaError_t layout_clear(const LayoutArgs &a, cudaStream_t s);
 // Outputs of an empty token set.
 cudaError_t layout_empty(const moe_layout &L, int R, int rpg, int mode, cudaStream_t s);
-// The place kernel, once the count phase (totals, segment offsets, cleared
-// scan state) is complete.
-cudaError_t launch_layout_place(const LayoutArgs &a, const DeviceCtx &ctx, cudaStream_t s);
+// Largest co-resident grid of a kernel with this much dynamic shared memory.
+cudaError_t max_resident_blocks(const void *kernel, size_t smem, const DeviceCtx &ctx, int &blocks);
 
 }  // namespace layout
 }  // namespace moe

@@ -157,7 +157,9 @@ MOE_API size_t moe_layout_workspace_size(int32_t T, int32_t k, int32_t E, int32_
                                  int32_t ranks_per_group, int32_t mode);
 
 /*
- * Stable per-destination row layout (count kernel + decoupled-lookback scan).
+ * Stable per-destination row layout (one cooperative launch: per-block bin
+ * counts, a bounded grid barrier, then each block's prefix from the count
+ * table and its rows).
  * Sources: the AllToAll(-v) destination chunks of "METRO AllGather vs AllToAll
  * for MoE decode", sections "Work the 8-GPU payload example" and "Distinguish
  * METRO from backend names"; the single-send dispatcher of the ainewsletter
@@ -251,10 +253,10 @@ MOE_API int moe_combine(const void *y, int32_t dtype, int32_t H, const moe_layou
  * a single replica, the METRO assignment of "METRO AllGather vs AllToAll for
  * MoE decode" (sections "changes the routing information" and "Add the
  * expert-weight traffic term") has no choice to make, so each pick's
- * destination rank is known as soon as the pick is; one kernel routes the
- * tokens and counts the demand vector, the layout's bins and the send matrix,
- * and the layout's place kernel follows.  Every output equals that of the
- * separate calls.
+ * destination rank is known as soon as the pick is; one cooperative kernel
+ * routes the tokens while counting the demand vector and the layout's bins,
+ * and after its grid barrier writes the layout's rows and the send matrix.
+ * Every output equals that of the separate calls.
  * expert_rank [E]: rank of each expert's only replica (every entry in [0, R);
  * a pick of an expert outside it sets MOE_ERR_BAD_INPUT and is skipped).
  * counts [E] out: the demand vector.  rank_active [R] out, or NULL: activated
@@ -341,8 +343,9 @@ MOE_API const char *moe_status_string(int status);
 /*
  * Test hook for the bounded waits.  wait_limit_ns: limit of every device-side
  * wait started after this call (0 restores the default of one second).
- * layout_silent_tile: index of one layout scan tile that does not publish its
- * prefix (-1 = none), so that its successors' waits run out and report
+ * layout_silent_tile: index of one block of the layout launches (moe_build_layout
+ * and moe_route_layout_single_replica) that never arrives at the grid barrier
+ * (-1 = none), so that the other blocks' waits run out and report
  * MOE_ERR_TIMEOUT instead of hanging.  Host-side settings, read at launch.
  */
 MOE_API int moe_debug_set_wait(uint64_t wait_limit_ns, int32_t layout_silent_tile);
