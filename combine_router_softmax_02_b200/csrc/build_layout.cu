@@ -34,13 +34,15 @@ __global__ void __launch_bounds__(kTile) layout_kernel(LayoutArgs a, DeviceCtx c
   const int t0 = blockIdx.x * a.chunk, t1 = min(a.T, t0 + a.chunk);
   smem_init(a, P, sm);
 
-  // phase 1: the block's rows per bin
+  // phase 1: the block's rows per bin (a one-tile chunk keeps its picks,
+  // weights included, for phase 2)
+  const bool one_tile = t1 - t0 <= kTile;
   bool bad = false;
   int c[4] = {0, 0, 0, 0};
+  TokenPicks<KM> p;
   for (int base = t0; base < t1; base += kTile) {
     const int t = base + (int)threadIdx.x;
-    TokenPicks<KM> p;
-    load_picks<KM>(a, sm + P.er, t, t < t1, false, p, bad);
+    load_picks<KM>(a, sm + P.er, t, t < t1, one_tile, p, bad);
     count_tile<KM>(a, p, lane, sm + P.cnt, c);
   }
   flush_counts(a, lane, sm + P.cnt, c);
@@ -49,7 +51,7 @@ __global__ void __launch_bounds__(kTile) layout_kernel(LayoutArgs a, DeviceCtx c
   if (!grid_barrier(a, ctx, &s_flag)) return;
 
   // phase 2: offsets and rows
-  phase2<KM>(a, P, sm, t0, t1, ctx);
+  phase2<KM>(a, P, sm, t0, t1, ctx, one_tile ? &p : nullptr);
 }
 
 std::atomic<unsigned long long> g_smem_set[4];

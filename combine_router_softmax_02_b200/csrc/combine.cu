@@ -284,9 +284,7 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
 
 template <typename Tin, typename Tout, int KM>
 cudaError_t launch_two_hop3(const TwoHopArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
-  long blocks = ((long)a.T + kFaninWarps - 1) / kFaninWarps;
-  const long cap = (long)ctx.num_sms * 16;
-  if (blocks > cap) blocks = cap;
+  const long blocks = ((long)a.T + kFaninWarps - 1) / kFaninWarps;  // uncapped, as in pack
   two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
@@ -308,10 +306,10 @@ cudaError_t launch_two_hop1(const TwoHopArgs &a, int out_dtype, const DeviceCtx 
 
 template <typename Tin, typename Tout, int KM>
 cudaError_t launch3(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
-  long blocks = (a.n_items >= 0) ? ((long)a.n_items + kFaninWarps - 1) / kFaninWarps
-                                 : (long)ctx.num_sms * 8;
-  const long cap = (long)ctx.num_sms * 16;
-  if (blocks > cap) blocks = cap;
+  // one block per 8 items, uncapped (resident blocks read and write one
+  // advancing window); a device-side item count gets a grid-stride grid
+  const long blocks = (a.n_items >= 0) ? ((long)a.n_items + kFaninWarps - 1) / kFaninWarps
+                                       : (long)ctx.num_sms * 8;
   if (blocks <= 0) return cudaSuccess;
   fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
   return count_launch(cudaGetLastError());

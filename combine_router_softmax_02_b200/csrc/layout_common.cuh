@@ -279,7 +279,7 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
   for (int x = tid; x < Q * V; x += kTile) {
     const int q = x / V, v = x % V;
     int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
-#pragma unroll 4
+#pragma unroll 8
     for (int g = q; g < a.nblk; g += Q) {
       const int4 c = __ldcg(reinterpret_cast<const int4 *>(a.agg + (size_t)g * a.NBp) + v);
       tot.x += c.x; tot.y += c.y; tot.z += c.z; tot.w += c.w;
@@ -541,17 +541,22 @@ __device__ __forceinline__ void rows_pick_tile(const LayoutArgs &a, const SmemPl
   __syncthreads();
 }
 
-// Phase 2 of the block's chunk [t0, t1) once the barrier has passed.
+// Phase 2 of the block's chunk [t0, t1) once the barrier has passed.  `pre`:
+// the thread's picks (with weights) kept from phase 1 when the chunk is one
+// tile, else null (the picks are loaded again, tile by tile).
 template <int KM>
 __device__ __forceinline__ void phase2(const LayoutArgs &a, const SmemPlan &P, int *sm, int t0,
-                                       int t1, DeviceCtx ctx) {
+                                       int t1, DeviceCtx ctx, const TokenPicks<KM> *pre) {
   bases_from_counts(a, P, sm, ctx);
   bool over = false, bad = false;
   for (int base = t0; base < t1; base += kTile) {
     const int t = base + (int)threadIdx.x;
     const bool live = t < t1;
     TokenPicks<KM> p;
-    load_picks<KM>(a, sm + P.er, t, live, true, p, bad);
+    if (pre)
+      p = *pre;
+    else
+      load_picks<KM>(a, sm + P.er, t, live, true, p, bad);
     if (a.mode == MOE_LAYOUT_PER_PICK)
       rows_pick_tile<KM>(a, P, sm, p, t, live, over);
     else
