@@ -227,6 +227,20 @@ class Layout:
             raise MoeError("moe_layout_workspace_size", 1)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
 
+    def tokens(self, t0: int, t1: int) -> moe_layout:
+        """A copy of the C struct for the token range [t0, t1), as moe_pack and
+        moe_combine accept it: the token-indexed arrays start at token t0 and
+        T = t1 - t0; the row-indexed arrays are shared."""
+        if not 0 <= t0 <= t1 <= self.T:
+            raise ValueError(f"token range [{t0}, {t1}) outside [0, {self.T})")
+        s = moe_layout.from_buffer_copy(self.struct)
+        s.T = t1 - t0
+        if self.T > 0:
+            s.token_rows = self.struct.token_rows + t0 * self.k * 4
+            if self.mode == TWO_HOP:
+                s.token_groups = self.struct.token_groups + t0 * self.k * 4
+        return s
+
 
 def build_layout(topk_idx, topk_w, expert_rank, layout: Layout, stream=None) -> Layout:
     _need(topk_idx, torch.int32, "topk_idx", 2)
@@ -243,7 +257,21 @@ def build_layout(topk_idx, topk_w, expert_rank, layout: Layout, stream=None) -> 
 
 
 # ----------------------------------------------------------- pack/combine ----
-def pack(x: torch.Tensor, layout: Layout, packed=None, packed_hop1=None, stream=None):
+def _token_slice(layout: Layout, t: torch.Tensor, tokens, name: str):
+    """(struct, pointer) for the whole layout, or for a token range of it with
+    the pointer of the [T][H] tensor t moved to the range's first token."""
+    if t.shape[0] != layout.T:
+        raise ValueError(f"{name} must have the layout's {layout.T} token rows")
+    if tokens is None:
+        return layout.struct, _p(t)
+    t0, t1 = tokens
+    s = layout.tokens(t0, t1)
+    return s, _p(t) + t0 * t.shape[1] * t.element_size()
+
+
+def pack(x: torch.Tensor, layout: Layout, packed=None, packed_hop1=None, stream=None, tokens=None):
+    """tokens=(t0, t1): pack only that token range of x (the rows it fills are
+    the same as in a full call)."""
     if x.dtype not in _DT:
         raise TypeError("x must be float16, bfloat16 or float32")
     _need(x, x.dtype, "x", 2)
@@ -253,15 +281,17 @@ def pack(x: torch.Tensor, layout: Layout, packed=None, packed_hop1=None, stream=
         packed = torch.empty((max(L.capacity, 1), H), dtype=x.dtype, device=x.device)
     if L.mode == TWO_HOP and packed_hop1 is None:
         packed_hop1 = torch.empty((max(L.capacity_hop1, 1), H), dtype=x.dtype, device=x.device)
-    _check(lib().moe_pack(_p(x), _DT[x.dtype], H, ctypes.byref(L.struct), _p(packed),
+    st, xp = _token_slice(L, x, tokens, "x")
+    _check(lib().moe_pack(xp, _DT[x.dtype], H, ctypes.byref(st), _p(packed),
                           _p(packed_hop1), _stream(stream)), "moe_pack")
     return (packed, packed_hop1) if L.mode == TWO_HOP else packed
 
 
 def combine(y: torch.Tensor, layout: Layout, out=None, out_dtype=None, row_coef=None,
-            hop1_buf=None, stream=None, store_hop1: bool = True):
+            hop1_buf=None, stream=None, store_hop1: bool = True, tokens=None):
     """TWO_HOP: the group partials go to hop1_buf (allocated if None), or are
-    not stored at all with store_hop1=False."""
+    not stored at all with store_hop1=False.  tokens=(t0, t1): combine only that
+    token range into out[t0:t1]."""
     if y.dtype not in _DT:
         raise TypeError("y must be float16, bfloat16 or float32")
     _need(y, y.dtype, "y", 2)
@@ -277,7 +307,8 @@ def combine(y: torch.Tensor, layout: Layout, out=None, out_dtype=None, row_coef=
         hop1_buf = torch.empty((max(L.capacity_hop1, 1), H), dtype=y.dtype, device=y.device)
     if not store_hop1:
         hop1_buf = None
-    _check(lib().moe_combine(_p(y), _DT[y.dtype], H, ctypes.byref(L.struct), _p(row_coef), _p(out),
+    st, op = _token_slice(L, out, tokens, "out")
+    _check(lib().moe_combine(_p(y), _DT[y.dtype], H, ctypes.byref(st), _p(row_coef), op,
                              _DT[out_dtype], _p(hop1_buf), _stream(stream)), "moe_combine")
     return out
 

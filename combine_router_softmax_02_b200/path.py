@@ -7,7 +7,7 @@ the path with identity experts (the packed rows are the expert outputs).
 """
 from __future__ import annotations
 
-from typing import Optional
+from typing import Callable, Optional
 
 import torch
 
@@ -72,3 +72,93 @@ class DispatchCombine:
     def step(self, logits: torch.Tensor, x: torch.Tensor) -> torch.Tensor:
         self.dispatch(logits, x)
         return self.combine()
+
+
+class HostPipeline:
+    """Steps of a DispatchCombine whose inputs and outputs are pinned host
+    buffers, with the host<->device copies overlapped with the kernels.
+
+    Three streams: copies in, kernels, copies out.  A step's logits are copied
+    first (the router needs nothing else); its activations follow in `chunks`
+    token ranges, and pack runs on each range as soon as it has arrived.  After
+    the experts (``experts(dc) -> y``, identity by default: y = the packed
+    rows), combine runs range by range and each finished range of the output
+    is copied back at once.  Device logits, activations and outputs are
+    double-buffered, so step s+1's copies in run while step s computes and
+    copies out; in steady state a step costs about the larger of its two copy
+    directions.  Every kernel is the DispatchCombine's (pack and combine on
+    token ranges give the rows and outputs of whole-range calls).
+    """
+
+    def __init__(self, dc: DispatchCombine, chunks: int = 8):
+        self.dc = dc
+        dev = dc.out.device
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_k = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        T, E, H = dc.T, dc.E, dc.H
+        self.logits = [torch.empty((T, E), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.x = [torch.empty((T, H), dtype=dc.dtype, device=dev) for _ in range(2)]
+        self.out = [torch.empty((T, H), dtype=dc.out_dtype, device=dev) for _ in range(2)]
+        n = max(1, min(chunks, T))
+        edges = [T * i // n for i in range(n + 1)]
+        self.ranges = [(a, b) for a, b in zip(edges, edges[1:]) if b > a]
+        self.in_free = [None, None]   # kernels done with logits[b] and x[b]
+        self.out_free = [None, None]  # copies out done with out[b]
+        self.last = [None, None, None]  # last event of each stream
+        self.i = 0
+
+    def _record(self, stream) -> torch.cuda.Event:
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        return ev
+
+    def wait(self, event: torch.cuda.Event):
+        """Every pipeline stream waits for `event` (work enqueued later starts after it)."""
+        for s in (self.s_in, self.s_k, self.s_out):
+            s.wait_event(event)
+
+    def join(self, stream=None):
+        """`stream` (default: the current one) waits for all enqueued pipeline work."""
+        stream = torch.cuda.current_stream() if stream is None else stream
+        for s in (self.s_in, self.s_k, self.s_out):
+            stream.wait_event(self._record(s))
+
+    def step(self, logits_h: torch.Tensor, x_h: torch.Tensor, out_h: torch.Tensor,
+             experts: Optional[Callable[[DispatchCombine], torch.Tensor]] = None):
+        """Enqueues one step: logits_h [T][E] f32, x_h [T][H] and out_h [T][H]
+        pinned host tensors.  out_h is complete once join() has been waited on."""
+        dc, b = self.dc, self.i & 1
+        self.i += 1
+        with torch.cuda.stream(self.s_in):
+            if self.in_free[b] is not None:
+                self.s_in.wait_event(self.in_free[b])
+            self.logits[b].copy_(logits_h, non_blocking=True)
+            ev_lg = self._record(self.s_in)
+            ev_x = []
+            for a, e in self.ranges:
+                self.x[b][a:e].copy_(x_h[a:e], non_blocking=True)
+                ev_x.append(self._record(self.s_in))
+        with torch.cuda.stream(self.s_k):
+            self.s_k.wait_event(ev_lg)
+            dc.route(self.logits[b])
+            for (a, e), ev in zip(self.ranges, ev_x):
+                self.s_k.wait_event(ev)
+                B.pack(self.x[b], dc.layout, dc.packed, dc.packed_hop1, tokens=(a, e))
+            self.in_free[b] = self._record(self.s_k)
+            y = dc.packed if experts is None else experts(dc)
+            if self.out_free[b] is not None:
+                self.s_k.wait_event(self.out_free[b])
+            ev_o = []
+            for a, e in self.ranges:
+                B.combine(y, dc.layout, self.out[b], dc.out_dtype, None, dc.hop1_buf, tokens=(a, e))
+                ev_o.append(self._record(self.s_k))
+        with torch.cuda.stream(self.s_out):
+            for (a, e), ev in zip(self.ranges, ev_o):
+                self.s_out.wait_event(ev)
+                out_h[a:e].copy_(self.out[b][a:e], non_blocking=True)
+            self.out_free[b] = self._record(self.s_out)
+
+    def synchronize(self):
+        for s in (self.s_in, self.s_k, self.s_out):
+            s.synchronize()

@@ -225,6 +225,11 @@ MOE_API int moe_build_layout_static(const int32_t *topk_idx, const float *topk_w
  * [capacity_hop1][H] receives the hop-1 (group) rows and packed the hop-2
  * (rank) rows, which equal the group rows they are forwarded from; both are
  * written from one read of each token.  packed_hop1 is ignored otherwise.
+ * Token ranges: pack reads only layout->T, k, mode, capacities, token_rows and
+ * token_groups (rows [0, T) of each) and writes absolute rows, so a copy of the
+ * layout with T = t1 - t0 and token_rows / token_groups advanced by t0 * k,
+ * given x advanced by t0 rows, packs tokens [t0, t1) exactly as a whole call
+ * would; calls on disjoint ranges may run in any order.
  */
 MOE_API int moe_pack(const void *x, int32_t dtype, int32_t H, const moe_layout *layout,
              void *packed, void *packed_hop1, moe_stream_t stream);
@@ -242,6 +247,9 @@ MOE_API int moe_pack(const void *x, int32_t dtype, int32_t H, const moe_layout *
  * rounded group partials in ascending group order.  hop1_buf [capacity_hop1][H]
  * of `dtype` receives the group partials at their hop-1 rows, or is NULL to
  * skip storing them.  hop1_buf is ignored for the other modes.
+ * Token ranges as for moe_pack: a layout copy with T = t1 - t0 and token_rows
+ * advanced by t0 * k, with out advanced by t0 rows, combines tokens [t0, t1)
+ * (row_coef, hop2_src_row and the row buffers are indexed by absolute row).
  */
 MOE_API int moe_combine(const void *y, int32_t dtype, int32_t H, const moe_layout *layout,
                 const float *row_coef, void *out, int32_t out_dtype, void *hop1_buf,
