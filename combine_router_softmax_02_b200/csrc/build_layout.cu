@@ -24,7 +24,7 @@ namespace moe {
 namespace layout {
 namespace {
 
-template <int KM>
+template <int KM, int MODE>
 __global__ void __launch_bounds__(kTile) layout_kernel(LayoutArgs a, DeviceCtx ctx) {
   extern __shared__ int4 smem_raw[];
   int *sm = reinterpret_cast<int *>(smem_raw);
@@ -35,33 +35,34 @@ __global__ void __launch_bounds__(kTile) layout_kernel(LayoutArgs a, DeviceCtx c
   smem_init(a, P, sm);
 
   // phase 1: the block's rows per bin (a one-tile chunk keeps its picks,
-  // weights included, for phase 2)
+  // weights included, and its ballots for phase 2)
   const bool one_tile = t1 - t0 <= kTile;
   bool bad = false;
   int c[4] = {0, 0, 0, 0};
   TokenPicks<KM> p;
+  Ballots bl{0u, 0u, 0u, 0u};
   for (int base = t0; base < t1; base += kTile) {
     const int t = base + (int)threadIdx.x;
-    load_picks<KM>(a, sm + P.er, t, t < t1, one_tile, p, bad);
-    count_tile<KM>(a, p, lane, sm + P.cnt, c);
+    load_picks<KM, MODE>(a, sm + P.er, t, t < t1, one_tile, p, bad);
+    count_tile<KM, MODE>(a, p, t < t1, lane, sm + P.cnt, c, bl);
   }
-  flush_counts(a, lane, sm + P.cnt, c);
+  flush_counts<MODE>(a, lane, sm + P.cnt, c);
   if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
   publish_counts(a, P, sm);
   if (!grid_barrier(a, ctx, &s_flag)) return;
 
   // phase 2: offsets and rows
-  phase2<KM>(a, P, sm, t0, t1, ctx, one_tile ? &p : nullptr);
+  phase2<KM, MODE>(a, P, sm, t0, t1, ctx, one_tile ? &p : nullptr, one_tile ? &bl : nullptr);
 }
 
-std::atomic<unsigned long long> g_smem_set[4];
+std::atomic<unsigned long long> g_smem_set[4][3];
 
-template <int KM>
+template <int KM, int MODE>
 cudaError_t launch_k(const LayoutArgs &a0, int kind, const DeviceCtx &ctx, cudaStream_t s) {
   LayoutArgs a = a0;
   const size_t smem = sizeof(int) * (size_t)smem_plan(a.E, a.NBp, a.R, false).total;
-  auto kern = layout_kernel<KM>;
-  cudaError_t err = set_smem_limit_once(kern, 200 * 1024, g_smem_set[kind]);
+  auto kern = layout_kernel<KM, MODE>;
+  cudaError_t err = set_smem_limit_once(kern, 200 * 1024, g_smem_set[kind][MODE]);
   if (err != cudaSuccess) return err;
   int resident = 0;
   if ((err = max_resident_blocks((const void *)kern, smem, ctx, resident)) != cudaSuccess) return err;
@@ -72,6 +73,13 @@ cudaError_t launch_k(const LayoutArgs &a0, int kind, const DeviceCtx &ctx, cudaS
   err = cudaLaunchCooperativeKernel((const void *)kern, dim3(a.nblk), dim3(kTile), args, smem, s);
   if (err != cudaSuccess) return err;
   return count_launch(cudaGetLastError());
+}
+
+template <int KM>
+cudaError_t launch_km(const LayoutArgs &a, int kind, const DeviceCtx &ctx, cudaStream_t s) {
+  if (a.mode == MOE_LAYOUT_PER_PICK) return launch_k<KM, MOE_LAYOUT_PER_PICK>(a, kind, ctx, s);
+  if (a.mode == MOE_LAYOUT_TWO_HOP) return launch_k<KM, MOE_LAYOUT_TWO_HOP>(a, kind, ctx, s);
+  return launch_k<KM, MOE_LAYOUT_DEDUP>(a, kind, ctx, s);
 }
 
 }  // namespace
@@ -140,10 +148,10 @@ cudaError_t launch_build_layout(const int *idx, const float *w, const int *exper
   if (T == 0) return layout::layout_empty(L, R, rpg, mode, s);
   const layout::LayoutArgs a =
       layout::make_layout_args(idx, w, expert_rank, T, tokens_per_rank, k, E, R, rpg, mode, L, ws);
-  if (k <= 2) return layout::launch_k<2>(a, 0, ctx, s);
-  if (k <= 4) return layout::launch_k<4>(a, 1, ctx, s);
-  if (k <= 8) return layout::launch_k<8>(a, 2, ctx, s);
-  return layout::launch_k<16>(a, 3, ctx, s);
+  if (k <= 2) return layout::launch_km<2>(a, 0, ctx, s);
+  if (k <= 4) return layout::launch_km<4>(a, 1, ctx, s);
+  if (k <= 8) return layout::launch_km<8>(a, 2, ctx, s);
+  return layout::launch_km<16>(a, 3, ctx, s);
 }
 
 }  // namespace moe

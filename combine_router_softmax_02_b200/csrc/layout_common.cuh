@@ -75,7 +75,7 @@ struct TokenPicks {
   unsigned long long gmask;  // groups of the token (TWO_HOP)
 };
 
-template <int KM>
+template <int KM, int MODE>
 __device__ __forceinline__ void load_picks(const LayoutArgs &a, const int *s_er, int t, bool live,
                                            bool want_w, TokenPicks<KM> &p, bool &bad) {
   p.present = 0;
@@ -105,7 +105,7 @@ __device__ __forceinline__ void load_picks(const LayoutArgs &a, const int *s_er,
       }
     }
   }
-  if (a.mode == MOE_LAYOUT_PER_PICK) {  // the row order needs distinct experts per token
+  if (MODE == MOE_LAYOUT_PER_PICK) {  // the row order needs distinct experts per token
 #pragma unroll
     for (int i = 0; i < KM; ++i)
 #pragma unroll
@@ -189,36 +189,52 @@ __device__ __forceinline__ void warp_merge(const TokenPicks<KM> &p, F &&f) {
 }
 
 // ------------------------------------------------------------- phase 1 ----
+// One warp's ballots of the mask bins: lane i holds those of ranks i, i + 32
+// (b0, b1) and of groups i, i + 32 (g0, g1).
+struct Ballots {
+  unsigned b0, b1, g0, g1;
+};
+
+// The warp's ballots of its tokens' ranks (and groups); a warp with no live
+// token skips the ballots (all zero).
+template <int MODE>
+__device__ __forceinline__ Ballots mask_ballots(const LayoutArgs &a, unsigned long long dmask,
+                                                unsigned long long gmask, bool live, int lane) {
+  Ballots bl{0u, 0u, 0u, 0u};
+  if (!__any_sync(kFull, live)) return bl;
+  warp_bin_ballots(dmask, a.R, lane, bl.b0, bl.b1);
+  if (MODE == MOE_LAYOUT_TWO_HOP) warp_bin_ballots(gmask, a.G, lane, bl.g0, bl.g1);
+  return bl;
+}
+
 // Adds one tile's bin counts of this warp into lane-held totals: c[0], c[1]
 // for ranks lane and lane + 32, c[2], c[3] for groups lane and lane + 32
-// (mask modes); experts go straight to the block counts (PER_PICK).
-template <int KM>
-__device__ __forceinline__ void count_tile(const LayoutArgs &a, const TokenPicks<KM> &p, int lane,
-                                           int *s_cnt, int (&c)[4]) {
-  if (a.mode == MOE_LAYOUT_PER_PICK) {
+// (mask modes; the tile's ballots are returned in bl); experts go straight
+// to the block counts (PER_PICK).
+template <int KM, int MODE>
+__device__ __forceinline__ void count_tile(const LayoutArgs &a, const TokenPicks<KM> &p, bool live,
+                                           int lane, int *s_cnt, int (&c)[4], Ballots &bl) {
+  if (MODE == MOE_LAYOUT_PER_PICK) {
     warp_merge<KM>(p, [&](uint32_t b, bool, unsigned ball, int, uint32_t) {
       if (lane == 0) atomicAdd(&s_cnt[b & 1023u], __popc(ball));
     });
     return;
   }
-  unsigned b0, b1;
-  warp_bin_ballots(p.dmask, a.R, lane, b0, b1);
-  c[0] += __popc(b0);
-  c[1] += __popc(b1);
-  if (a.mode == MOE_LAYOUT_TWO_HOP) {
-    warp_bin_ballots(p.gmask, a.G, lane, b0, b1);
-    c[2] += __popc(b0);
-    c[3] += __popc(b1);
-  }
+  bl = mask_ballots<MODE>(a, p.dmask, p.gmask, live, lane);
+  c[0] += __popc(bl.b0);
+  c[1] += __popc(bl.b1);
+  c[2] += __popc(bl.g0);
+  c[3] += __popc(bl.g1);
 }
 
 // Moves the lane-held mask-bin totals into the block counts.
+template <int MODE>
 __device__ __forceinline__ void flush_counts(const LayoutArgs &a, int lane, int *s_cnt,
                                              const int (&c)[4]) {
-  if (a.mode == MOE_LAYOUT_PER_PICK) return;
+  if (MODE == MOE_LAYOUT_PER_PICK) return;
   if (lane < a.R && c[0]) atomicAdd(&s_cnt[lane], c[0]);
   if (lane + 32 < a.R && c[1]) atomicAdd(&s_cnt[lane + 32], c[1]);
-  if (a.mode == MOE_LAYOUT_TWO_HOP) {
+  if (MODE == MOE_LAYOUT_TWO_HOP) {
     if (lane < a.G && c[2]) atomicAdd(&s_cnt[a.R + lane], c[2]);
     if (lane + 32 < a.G && c[3]) atomicAdd(&s_cnt[a.R + lane + 32], c[3]);
   }
@@ -269,6 +285,7 @@ __device__ __forceinline__ bool grid_barrier(const LayoutArgs &a, const DeviceCt
 // ------------------------------------------------------------- phase 2 ----
 // Per-bin totals (into s_cnt) and this block's base (into s_base) from the
 // count table, then the segment offsets; block 0 writes the layout's offsets.
+template <int MODE>
 __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const SmemPlan &P, int *sm,
                                                   DeviceCtx ctx) {
   const int tid = threadIdx.x;
@@ -309,7 +326,7 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
   const int *s_er = sm + P.er;
   const moe_layout &L = a.L;
   const int lane = tid & 31;
-  if (a.mode == MOE_LAYOUT_PER_PICK) {
+  if (MODE == MOE_LAYOUT_PER_PICK) {
     if (tid < a.R) {  // each rank walks its experts in ascending order
       int run = 0;
       for (int e = 0; e < a.E; ++e)
@@ -352,7 +369,7 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
     }
   } else if (tid < 32) {
     // exclusive scans of the rank totals and of the group totals (<= 64 each)
-    for (int part = 0; part < (a.mode == MOE_LAYOUT_TWO_HOP ? 2 : 1); ++part) {
+    for (int part = 0; part < (MODE == MOE_LAYOUT_TWO_HOP ? 2 : 1); ++part) {
       const int n = part ? a.G : a.R, off = part ? a.R : 0;
       const int v0 = lane < n ? s_cnt[off + lane] : 0, v1 = lane + 32 < n ? s_cnt[off + lane + 32] : 0;
       int i0 = v0, i1 = v1;
@@ -392,20 +409,19 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
 
 // Rows of one tile of mask-bin tokens (DEDUP, TWO_HOP).  Every thread of the
 // block calls it; `t` is the thread's token, `live` whether it has one.
-template <int KM>
+template <int KM, int MODE>
 __device__ __forceinline__ void rows_mask_tile(const LayoutArgs &a, const SmemPlan &P, int *sm,
-                                               const TokenPicks<KM> &p, int t, bool live, bool &over) {
+                                               const TokenPicks<KM> &p, const Ballots &bl, int t,
+                                               bool live, bool &over) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int *s_w = sm + P.w + warp * a.NBp;
   const int *s_woff = sm + P.woff + warp * a.NBp;
-  unsigned b0, b1, g0 = 0, g1 = 0;
-  warp_bin_ballots(p.dmask, a.R, lane, b0, b1);
+  const unsigned b0 = bl.b0, b1 = bl.b1;
   if (lane < a.R) s_w[lane] = b0;
   if (lane + 32 < a.R) s_w[lane + 32] = b1;
-  if (a.mode == MOE_LAYOUT_TWO_HOP) {
-    warp_bin_ballots(p.gmask, a.G, lane, g0, g1);
-    if (lane < a.G) s_w[a.R + lane] = g0;
-    if (lane + 32 < a.G) s_w[a.R + lane + 32] = g1;
+  if (MODE == MOE_LAYOUT_TWO_HOP) {
+    if (lane < a.G) s_w[a.R + lane] = bl.g0;
+    if (lane + 32 < a.G) s_w[a.R + lane + 32] = bl.g1;
   }
   // send counts: source rank of the token -> its ranks
   int *s_send = sm + P.send;
@@ -435,7 +451,7 @@ __device__ __forceinline__ void rows_mask_tile(const LayoutArgs &a, const SmemPl
   const unsigned lt = lanemask_lt();
   const size_t tk = (size_t)t * a.k;
   auto row_of = [&](int bin) { return s_woff[bin] + __popc((unsigned)s_w[bin] & lt); };
-  if (a.mode == MOE_LAYOUT_TWO_HOP) {
+  if (MODE == MOE_LAYOUT_TWO_HOP) {
     int cg = 0;
     for (unsigned long long m = p.gmask; m; m &= m - 1, ++cg) {
       const int g = __ffsll((long long)m) - 1;
@@ -470,7 +486,7 @@ __device__ __forceinline__ void rows_mask_tile(const LayoutArgs &a, const SmemPl
       L.token_rows[tk + c] = -1;
       over = true;
     }
-    if (a.mode == MOE_LAYOUT_TWO_HOP) {
+    if (MODE == MOE_LAYOUT_TWO_HOP) {
       const int g = r / a.rpg;
       int row1 = row_of(a.R + g);
       if (row1 >= L.capacity_hop1) row1 = -1;
@@ -541,14 +557,17 @@ __device__ __forceinline__ void rows_pick_tile(const LayoutArgs &a, const SmemPl
   __syncthreads();
 }
 
-// Phase 2 of the block's chunk [t0, t1) once the barrier has passed.  `pre`:
-// the thread's picks (with weights) kept from phase 1 when the chunk is one
-// tile, else null (the picks are loaded again, tile by tile).
-template <int KM>
+// Phase 2 of the block's chunk [t0, t1) once the barrier has passed.  `pre`
+// and `pre_bl`: the thread's picks (with weights) and its warp's ballots kept
+// from phase 1 when the chunk is one tile, else null (loaded again, tile by
+// tile).
+template <int KM, int MODE>
 __device__ __forceinline__ void phase2(const LayoutArgs &a, const SmemPlan &P, int *sm, int t0,
-                                       int t1, DeviceCtx ctx, const TokenPicks<KM> *pre) {
-  bases_from_counts(a, P, sm, ctx);
+                                       int t1, DeviceCtx ctx, const TokenPicks<KM> *pre,
+                                       const Ballots *pre_bl) {
+  bases_from_counts<MODE>(a, P, sm, ctx);
   bool over = false, bad = false;
+  const int lane = threadIdx.x & 31;
   for (int base = t0; base < t1; base += kTile) {
     const int t = base + (int)threadIdx.x;
     const bool live = t < t1;
@@ -556,11 +575,13 @@ __device__ __forceinline__ void phase2(const LayoutArgs &a, const SmemPlan &P, i
     if (pre)
       p = *pre;
     else
-      load_picks<KM>(a, sm + P.er, t, live, true, p, bad);
-    if (a.mode == MOE_LAYOUT_PER_PICK)
+      load_picks<KM, MODE>(a, sm + P.er, t, live, true, p, bad);
+    if (MODE == MOE_LAYOUT_PER_PICK) {
       rows_pick_tile<KM>(a, P, sm, p, t, live, over);
-    else
-      rows_mask_tile<KM>(a, P, sm, p, t, live, over);
+    } else {
+      const Ballots bl = pre_bl ? *pre_bl : mask_ballots<MODE>(a, p.dmask, p.gmask, live, lane);
+      rows_mask_tile<KM, MODE>(a, P, sm, p, bl, t, live, over);
+    }
   }
   if (over) set_status(ctx.status, MOE_ERR_CAPACITY);
   // the block's send counts (send_counts was cleared before the barrier)

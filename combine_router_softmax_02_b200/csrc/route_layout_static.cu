@@ -84,7 +84,13 @@ __global__ void __launch_bounds__(kTile) route_layout_kernel(RouteArgs ra, Layou
   if (!layout::grid_barrier(a, ctx, &s_flag)) return;
 
   // phase 2: the layout's offsets and rows, then the demand vector
-  layout::phase2<KM>(a, P, sm, t0, t1, ctx, static_cast<const layout::TokenPicks<KM> *>(nullptr));
+  using Picks = layout::TokenPicks<KM>;
+  if (a.mode == MOE_LAYOUT_DEDUP)
+    layout::phase2<KM, MOE_LAYOUT_DEDUP>(a, P, sm, t0, t1, ctx, (const Picks *)nullptr, nullptr);
+  else if (a.mode == MOE_LAYOUT_TWO_HOP)
+    layout::phase2<KM, MOE_LAYOUT_TWO_HOP>(a, P, sm, t0, t1, ctx, (const Picks *)nullptr, nullptr);
+  else
+    layout::phase2<KM, MOE_LAYOUT_PER_PICK>(a, P, sm, t0, t1, ctx, (const Picks *)nullptr, nullptr);
   for (int i = tid; i < a.E; i += kTile)
     if (s_hist[i]) atomicAdd(&ra.counts[i], s_hist[i]);
   if (!ra.rank_active) return;
