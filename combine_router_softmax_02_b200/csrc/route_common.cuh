@@ -31,12 +31,13 @@ namespace route {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-// Monotone map float -> uint32 (larger float, larger key); -0 and +0 map to
-// the same key so they tie like the floats compare.  Finite values map into
-// [0x00800000, 0xff800000); -inf, +inf and NaNs land outside that range.
+// Monotone map float -> uint32 (larger float, larger key): negative values
+// have all bits flipped, the others their sign bit set.  Adding +0 first turns
+// -0 into +0, so the two zeros tie like the floats compare.  Finite values map
+// into [0x00800000, 0xff800000); -inf, +inf and NaNs land outside that range.
 __device__ __forceinline__ uint32_t order_key(float v) {
-  uint32_t u = (v == 0.0f) ? 0u : __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
 }
 
 // Inverse of order_key (a zero key comes back as +0).
@@ -82,7 +83,8 @@ struct Lanes {
 
 // Routes the token whose logits start at `row`.  Lanes r < k return pick r in
 // (my_e, my_w); `bad` is set on lanes that saw a non-finite logit.  s_ck and
-// s_ce are this warp's 32-entry shared-memory candidate buffers.
+// s_ce are this warp's 32-entry shared-memory candidate buffers (s_ck
+// 16-byte aligned).
 template <int EPL, bool FULL>
 __device__ __forceinline__ void route_token(const float *row, int E, int k, int n_groups, int gpt,
                                             int renorm, const Lanes<EPL, FULL> &L, uint32_t *s_ck,
@@ -148,7 +150,7 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
   for (int r = 0; r < k; ++r) {
     tau = (r == 0 && fresh) ? top : __reduce_max_sync(kFull, lm);
     const unsigned b = __ballot_sync(kFull, lm == tau);
-    if (lane == __ffs(b) - 1) lm = 0;
+    if (lane == 31 - __clz(b)) lm = 0;  // any one lane holding the value
   }
 
   // compaction in ascending expert order: slot j of lane l is expert l + 32 j
@@ -169,13 +171,18 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
   my_e = 0;
   uint32_t my_k = 0;
   if (total <= 32) {
+    // zero keys pad the candidates to a multiple of 4: they beat no candidate
+    if (lane >= (int)total && lane < (int)((total + 3) & ~3u)) s_ck[lane] = 0u;
     __syncwarp();
     const uint32_t ck = lane < (int)total ? s_ck[lane] : 0u;
     const int ce = lane < (int)total ? s_ce[lane] : 0;
     int rank = 0;
-    for (int j = 0; j < (int)total; ++j) {
-      const uint32_t kj = s_ck[j];  // broadcast
-      rank += (kj > ck || (kj == ck && j < lane)) ? 1 : 0;
+    for (int j = 0; j < (int)total; j += 4) {
+      const uint4 q = *reinterpret_cast<const uint4 *>(s_ck + j);  // broadcast
+      rank += (q.x > ck || (q.x == ck && j < lane)) ? 1 : 0;
+      rank += (q.y > ck || (q.y == ck && j + 1 < lane)) ? 1 : 0;
+      rank += (q.z > ck || (q.z == ck && j + 2 < lane)) ? 1 : 0;
+      rank += (q.w > ck || (q.w == ck && j + 3 < lane)) ? 1 : 0;
     }
     __syncwarp();
     if (lane < (int)total && rank < k) {

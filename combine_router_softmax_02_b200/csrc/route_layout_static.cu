@@ -34,7 +34,7 @@ template <int EPL, bool FULL, int KM>
 __global__ void __launch_bounds__(kTile) route_layout_kernel(RouteArgs ra, LayoutArgs a, DeviceCtx ctx) {
   extern __shared__ int4 smem_raw[];
   int *sm = reinterpret_cast<int *>(smem_raw);
-  __shared__ uint32_t s_ck[kWarps][32];
+  __shared__ __align__(16) uint32_t s_ck[kWarps][32];
   __shared__ int s_ce[kWarps][32];
   __shared__ int s_flag;
   const SmemPlan P = layout::smem_plan(a.E, a.NBp, a.R, true);

@@ -9,7 +9,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          int E, int k, int n_groups, int gpt,
                                                          int renorm, int *__restrict__ idx_out,
                                                          float *__restrict__ w_out, DeviceCtx ctx) {
-  __shared__ uint32_t s_ck[8][32];  // per-warp candidate keys
+  __shared__ __align__(16) uint32_t s_ck[8][32];  // per-warp candidate keys
   __shared__ int s_ce[8][32];       // and their experts
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
