@@ -35,6 +35,8 @@ struct FaninArgs {
   const float *coef;        // per source row; nullptr = 1
   int src_cap;              // rows in y
   int nvec;                 // 16-byte input vectors per row
+  int slices;               // warps per item, each a column slice of the row
+  int svec;                 // 16-byte input vectors per slice
 };
 
 template <typename T>
@@ -128,8 +130,12 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
   SrcEntry *tab = s_tab[warp];
   int n = a.n_items;
   if (n < 0) n = min(max(*a.n_items_dev, 0), a.cap_items);
+  const int n_work = n * a.slices;  // < 2^31: slices > 1 only for few rows
   bool bounds = false;
-  for (int item = blockIdx.x * kFaninWarps + warp; item < n; item += gridDim.x * kFaninWarps) {
+  for (unsigned wk = blockIdx.x * kFaninWarps + warp; wk < (unsigned)n_work; wk += gridDim.x * kFaninWarps) {
+    const int item = (int)(wk / (unsigned)a.slices);
+    const int vbeg = (int)(wk % (unsigned)a.slices) * a.svec;
+    const int vend = min(a.nvec, vbeg + a.svec);
     int my_r = -1;
     float my_c = 0.0f;
     if (lane < a.k) {
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
     }
     __syncwarp();
     uint8_t *orow = a.out + (size_t)item * a.rb_out;
-    for (int v = lane; v < a.nvec; v += 32) {
+    for (int v = vbeg + lane; v < vend; v += 32) {
       uint4 d[KM];
 #pragma unroll
       for (int j = 0; j < KM; ++j)
@@ -198,6 +204,7 @@ struct TwoHopArgs {
   const float *coef;
   int cap, cap1;
   int nvec;
+  int slices, svec;         // column slices per token, vectors per slice
 };
 
 // TWO_HOP reverse in one pass per token, one warp per token: the token's rank
@@ -215,7 +222,11 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
   const int warp = threadIdx.x >> 5;
   SrcEntry *tab = s_tab[warp];
   bool bounds = false;
-  for (int t = blockIdx.x * kFaninWarps + warp; t < a.T; t += gridDim.x * kFaninWarps) {
+  const int n_work = a.T * a.slices;  // < 2^31: slices > 1 only for few rows
+  for (unsigned wk = blockIdx.x * kFaninWarps + warp; wk < (unsigned)n_work; wk += gridDim.x * kFaninWarps) {
+    const int t = (int)(wk / (unsigned)a.slices);
+    const int vbeg = (int)(wk % (unsigned)a.slices) * a.svec;
+    const int vend = min(a.nvec, vbeg + a.svec);
     int my_r = -1, my_s = -1;
     float my_c = 0.0f;
     if (lane < a.k) {
@@ -248,7 +259,7 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
     }
     __syncwarp();
     uint8_t *orow = a.out + (size_t)t * a.rb_out;
-    for (int v = lane; v < a.nvec; v += 32) {
+    for (int v = vbeg + lane; v < vend; v += 32) {
       uint4 d[KM];
 #pragma unroll
       for (int j = 0; j < KM; ++j)
@@ -284,7 +295,7 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
 
 template <typename Tin, typename Tout, int KM>
 cudaError_t launch_two_hop3(const TwoHopArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
-  const long blocks = ((long)a.T + kFaninWarps - 1) / kFaninWarps;  // uncapped, as in pack
+  const long blocks = ((long)a.T * a.slices + kFaninWarps - 1) / kFaninWarps;  // uncapped, as in pack
   two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
@@ -308,7 +319,7 @@ template <typename Tin, typename Tout, int KM>
 cudaError_t launch3(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   // one block per 8 items, uncapped (resident blocks read and write one
   // advancing window); a device-side item count gets a grid-stride grid
-  const long blocks = (a.n_items >= 0) ? ((long)a.n_items + kFaninWarps - 1) / kFaninWarps
+  const long blocks = (a.n_items >= 0) ? ((long)a.n_items * a.slices + kFaninWarps - 1) / kFaninWarps
                                        : (long)ctx.num_sms * 8;
   if (blocks <= 0) return cudaSuccess;
   fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
@@ -360,6 +371,7 @@ cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
     a.coef = coef;
     a.src_cap = L.capacity;
     a.nvec = (int)(a.rb_in / 16);
+    row_slices(a.n_items, a.nvec, ctx.num_sms, a.slices, a.svec);
     return launch_fanin(a, dtype, out_dtype, ctx, s);
   }
   // both reverse hops in one pass per token
@@ -378,6 +390,7 @@ cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
   b.cap1 = L.capacity_hop1;
   b.nvec = (int)(b.rb_in / 16);
   if (b.T == 0) return cudaSuccess;
+  row_slices(b.T, b.nvec, ctx.num_sms, b.slices, b.svec);
   if (dtype == MOE_F16) return launch_two_hop1<__half>(b, out_dtype, ctx, s);
   if (dtype == MOE_BF16) return launch_two_hop1<__nv_bfloat16>(b, out_dtype, ctx, s);
   return launch_two_hop1<float>(b, out_dtype, ctx, s);

@@ -84,6 +84,23 @@ inline cudaError_t set_smem_limit_once(Kern kern, int bytes, std::atomic<unsigne
   return e;
 }
 
+// Column slices per row for the one-warp-per-row copy kernels: few rows (the
+// decode regime) would leave most SMs idle and each warp walking its whole row
+// one dependent round trip after another, so a row is split into slices of
+// whole warp-widths (32 16-byte vectors each) until there are about 32 warps
+// per SM; many rows keep one slice each.
+inline void row_slices(long rows, int nvec, int num_sms, int &slices, int &svec) {
+  const long want = (long)num_sms * 32;
+  long s = rows > 0 ? (want + rows - 1) / rows : 1;
+  const long cap = nvec / 32 > 0 ? nvec / 32 : 1;
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  svec = (int)((((long)nvec + s - 1) / s + 31) / 32 * 32);
+  if (svec < 1) svec = 1;
+  slices = (nvec + svec - 1) / svec;
+  if (slices < 1) slices = 1;
+}
+
 // Host-side count of kernel launches (moe_kernel_launches); each launch site
 // calls count_launch() after a launch that cudaGetLastError() accepted.
 extern std::atomic<unsigned long long> g_kernel_launches;

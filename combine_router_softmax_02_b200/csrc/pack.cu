@@ -37,6 +37,8 @@ struct FanoutArgs {
   const int *lists[2];
   uint8_t *dst[2];
   int dst_cap[2];           // rows in dst[l]
+  int slices;               // warps per item, each a column slice of the row
+  int svec;                 // 16-byte vectors per slice
 };
 
 // Column vectors per lane per iteration (a sweep over 1-4 on both benchmark
@@ -54,8 +56,12 @@ __global__ void __launch_bounds__(256) fanout_kernel(FanoutArgs a, DeviceCtx ctx
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   const int nvec = (int)(a.rb / 16);
+  const int n_work = a.n_items * a.slices;  // < 2^31: slices > 1 only for few rows
   bool bounds = false;
-  for (int item = blockIdx.x * wpb + (threadIdx.x >> 5); item < a.n_items; item += gridDim.x * wpb) {
+  for (unsigned wk = blockIdx.x * wpb + (threadIdx.x >> 5); wk < (unsigned)n_work; wk += gridDim.x * wpb) {
+    const int item = (int)(wk / (unsigned)a.slices);
+    const int vbeg = (int)(wk % (unsigned)a.slices) * a.svec;
+    const int vend = min(nvec, vbeg + a.svec);
     int my = -1;
     if (lane < W) {
       const int l = lane / KM, j = lane % KM;
@@ -75,17 +81,17 @@ __global__ void __launch_bounds__(256) fanout_kernel(FanoutArgs a, DeviceCtx ctx
       dst[j] = a.dst[j / KM] + (size_t)(r < 0 ? 0 : r) * a.rb;
     }
     const uint8_t *srow = a.src + (size_t)item * a.rb;
-    for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
+    for (int v0 = vbeg + lane; v0 < vend; v0 += 32 * U) {
       uint4 x[U];
 #pragma unroll
       for (int u = 0; u < U; ++u)
-        if (v0 + 32 * u < nvec) x[u] = ld_stream_v4(srow + (size_t)(v0 + 32 * u) * 16);
+        if (v0 + 32 * u < vend) x[u] = ld_stream_v4(srow + (size_t)(v0 + 32 * u) * 16);
 #pragma unroll
       for (int j = 0; j < W; ++j)
         if (dmask >> j & 1u)
 #pragma unroll
           for (int u = 0; u < U; ++u)
-            if (v0 + 32 * u < nvec) st_v4(dst[j] + (size_t)(v0 + 32 * u) * 16, x[u]);
+            if (v0 + 32 * u < vend) st_v4(dst[j] + (size_t)(v0 + 32 * u) * 16, x[u]);
     }
   }
   if (bounds) set_status(ctx.status, MOE_ERR_BOUNDS);
@@ -94,7 +100,7 @@ __global__ void __launch_bounds__(256) fanout_kernel(FanoutArgs a, DeviceCtx ctx
 template <int KM, int NL>
 cudaError_t launch_kn(const FanoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   const int wpb = 8;
-  const long blocks = ((long)a.n_items + wpb - 1) / wpb;
+  const long blocks = ((long)a.n_items * a.slices + wpb - 1) / wpb;
   fanout_kernel<KM, NL, kU><<<(unsigned)blocks, wpb * 32, 0, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
@@ -107,8 +113,9 @@ cudaError_t launch_nl(const FanoutArgs &a, const DeviceCtx &ctx, cudaStream_t s)
   return launch_kn<16, NL>(a, ctx, s);
 }
 
-cudaError_t launch_fanout(const FanoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
+cudaError_t launch_fanout(FanoutArgs a, const DeviceCtx &ctx, cudaStream_t s) {
   if (a.n_items <= 0) return cudaSuccess;
+  row_slices(a.n_items, (int)(a.rb / 16), ctx.num_sms, a.slices, a.svec);
   return a.lists[1] ? launch_nl<2>(a, ctx, s) : launch_nl<1>(a, ctx, s);
 }
 
