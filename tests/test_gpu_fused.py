@@ -66,6 +66,19 @@ def test_fused_edges(moe, T, E, k, R, mode, rpg):
     assert_same_route(moe, cfg, sep, fus)
 
 
+@pytest.mark.parametrize("mode,rpg", [(W.DEDUP, 1), (W.TWO_HOP, 2)])
+def test_fused_multi_tile_chunks(moe, mode, rpg):
+    """140000 tokens: the fused launch's chunks span two tiles each (phase 2
+    reloads the picks its warps wrote in phase 1)."""
+    cfg = W.Config("mt", "mt", T=140000, R=8, H=64, dtype="bf16", E=64, k=2, mode=mode,
+                   ranks_per_group=rpg if mode == W.TWO_HOP else 0)
+    rng = np.random.default_rng(11)
+    logits = rng.standard_normal((cfg.T, cfg.E)).astype(np.float32)
+    er = rng.integers(0, cfg.R, size=cfg.E).astype(np.int32)
+    sep, fus = run_both(moe, cfg, logits, er)
+    assert_same_route(moe, cfg, sep, fus)
+
+
 def test_fused_full_path_two_hop_output(moe):
     """The whole two-hop path with the fused front end gives the same output bits."""
     cfg = W.CONFIGS["c5"].with_(T=4096)

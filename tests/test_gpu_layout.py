@@ -1,6 +1,7 @@
-"""GPU parity: the stable per-destination layout (count kernel + decoupled
-lookback scan) against the CPU oracle: every integer field bit-exact, the
-coefficients within their float bound; plus the device-side error paths."""
+"""GPU parity: the stable per-destination layout (one cooperative launch:
+per-block counts, grid barrier, each block's prefix from the count table)
+against the CPU oracle: every integer field bit-exact, the coefficients within
+their float bound; plus the device-side error paths."""
 import numpy as np
 import pytest
 import torch
@@ -42,6 +43,20 @@ def test_layout_full_size_configs(moe, name, mode, placement):
     L = run_layout(moe, idx, w, er, cfg.T, cfg.tokens_per_rank, cfg.k, cfg.E, cfg.R, mode, rpg)
     assert moe.get_status() == 0
     ref = ref_layout(idx, w, er, cfg.tokens_per_rank, cfg.R, mode, rpg)
+    assert_layout_equal(layout_fields(L, mode), ref, mode, w_tol=cfg.k * U)
+
+
+@pytest.mark.parametrize("mode,R,rpg", [(W.DEDUP, 32, 1), (W.PER_PICK, 32, 1), (W.TWO_HOP, 32, 4)])
+def test_layout_multi_tile_chunks(moe, mode, R, rpg):
+    """100000 tokens: each block's chunk spans two 256-token tiles, so phase 2
+    reloads the picks tile by tile and carries every bin's base across tiles."""
+    cfg = W.CONFIGS["c3"].with_(T=100000, R=R, mode=mode)
+    idx, w = oracle.route_topk(W.make_logits(cfg, 3), cfg.k)
+    er = np.random.default_rng(5).integers(0, R, size=cfg.E).astype(np.int32)
+    tpr = -(-cfg.T // R)
+    L = run_layout(moe, idx, w, er, cfg.T, tpr, cfg.k, cfg.E, R, mode, rpg)
+    assert moe.get_status() == 0
+    ref = ref_layout(idx, w, er, tpr, R, mode, rpg)
     assert_layout_equal(layout_fields(L, mode), ref, mode, w_tol=cfg.k * U)
 
 
