@@ -5,11 +5,12 @@
 // t's rows i, in ascending row order, of coef[i] * y[i], accumulated in
 // float32 and rounded to nearest-even into the output dtype.
 //
-// Generic fan-in, one warp per output row: the item's (<= k) source rows and
-// coefficients are broadcast from lanes 0..k-1, then each lane walks 16-byte
-// column vectors with all of the item's rows in flight at once
-// (ld.global.nc.L1::no_allocate), multiply-adds them in row order and writes
-// the result once.  No atomics: the result does not depend on scheduling.
+// Generic fan-in, one warp per output row (or column slice of it): the item's
+// (<= k) source rows and coefficients go to a per-warp table, then each lane
+// walks 16-byte column vectors, with the item's rows copied into shared memory
+// two vectors ahead (cp.async, two stages, so the loads overlap the
+// arithmetic and the store), multiply-adds them in row order and writes the
+// result once.  No atomics: the result does not depend on scheduling.
 // Items are tokens and lists token_rows.  The two-hop reverse has its own
 // kernel below (both hops in one pass per token).
 #include <cuda_bf16.h>
@@ -120,14 +121,28 @@ __device__ __forceinline__ SrcEntry read_entry(const SrcEntry *e) {
   return r;
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), and its group fences.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <typename Tin, typename Tout, int KM>
 __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
     fanin_kernel(FaninArgs a, DeviceCtx ctx) {
   constexpr int VE = Elem<Tin>::kPerVec;
+  extern __shared__ uint4 s_stage[];  // [warp][stage 2][KM][32 lanes]
   __shared__ __align__(16) SrcEntry s_tab[kFaninWarps][KM];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   SrcEntry *tab = s_tab[warp];
+  uint4 *stage = s_stage + (size_t)warp * 2 * KM * 32 + lane;  // slot (st, j): stage[(st * KM + j) * 32]
   int n = a.n_items;
   if (n < 0) n = min(max(*a.n_items_dev, 0), a.cap_items);
   const int n_work = n * a.slices;  // < 2^31: slices > 1 only for few rows
@@ -156,21 +171,33 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
       tab[lane] = e;
     }
     __syncwarp();
-    uint8_t *orow = a.out + (size_t)item * a.rb_out;
-    for (int v = vbeg + lane; v < vend; v += 32) {
-      uint4 d[KM];
+    auto issue = [&](int v, int st) {
 #pragma unroll
       for (int j = 0; j < KM; ++j)
-        if (vmask >> j & 1u) d[j] = ld_stream_v4((const uint8_t *)read_entry(tab + j).addr + (size_t)v * 16);
+        if (vmask >> j & 1u)
+          cp_async16(stage + (st * KM + j) * 32, (const uint8_t *)read_entry(tab + j).addr + (size_t)v * 16);
+      cp_async_commit();
+    };
+    uint8_t *orow = a.out + (size_t)item * a.rb_out;
+    int st = 0;
+    if (vbeg + lane < vend) issue(vbeg + lane, 0);
+    for (int v = vbeg + lane; v < vend; v += 32, st ^= 1) {
+      if (v + 32 < vend) {
+        issue(v + 32, st ^ 1);
+        cp_async_wait<1>();  // this vector's group is in
+      } else {
+        cp_async_wait<0>();
+      }
       float acc[VE];
 #pragma unroll
       for (int e = 0; e < VE; ++e) acc[e] = 0.0f;
 #pragma unroll
       for (int j = 0; j < KM; ++j)
         if (vmask >> j & 1u) {
+          const uint4 d = stage[(st * KM + j) * 32];
           const float c = read_entry(tab + j).coef;
 #pragma unroll
-          for (int e = 0; e < VE; ++e) acc[e] = fmaf(c, Elem<Tin>::get(d[j], e), acc[e]);
+          for (int e = 0; e < VE; ++e) acc[e] = fmaf(c, Elem<Tin>::get(d, e), acc[e]);
         }
       store_out<Tout, VE>(orow + (size_t)v * VE * sizeof(Tout), acc);
     }
@@ -207,20 +234,29 @@ struct TwoHopArgs {
   int slices, svec;         // column slices per token, vectors per slice
 };
 
-// TWO_HOP reverse in one pass per token, one warp per token: the token's rank
-// rows are summed group by group in float32 (ascending rows), each group
-// partial is rounded to the activation dtype (the slow-fabric wire format),
-// stored to its hop-1 row when a buffer is given, and the rounded partials are
-// summed in ascending group order into the token.  Bit-identical to running
-// the two reverse hops one after the other, without re-reading the partials.
+// TWO_HOP reverse in one pass per token, one warp per token (or column slice):
+// the token's rank rows are summed group by group in float32 (ascending rows),
+// each group partial is rounded to the activation dtype (the slow-fabric wire
+// format), stored to its hop-1 row when a buffer is given, and the rounded
+// partials are summed in ascending group order into the token.  Bit-identical
+// to running the two reverse hops one after the other, without re-reading the
+// partials.
+//
+// The rows' column vectors go through shared memory in two stages with
+// cp.async: while a lane works on vector v, its copies of vector v + 32 are in
+// flight, so the loads overlap the arithmetic and the stores without holding
+// registers.  Each lane reads back only the slots it copied itself, so the
+// per-thread wait_group is the only fence needed.
 template <typename Tin, typename Tout, int KM>
 __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
     two_hop_fanin_kernel(TwoHopArgs a, DeviceCtx ctx) {
   constexpr int VE = Elem<Tin>::kPerVec;
+  extern __shared__ uint4 s_stage[];  // [warp][stage 2][KM][32 lanes]
   __shared__ __align__(16) SrcEntry s_tab[kFaninWarps][KM];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   SrcEntry *tab = s_tab[warp];
+  uint4 *stage = s_stage + (size_t)warp * 2 * KM * 32 + lane;  // slot (st, j): stage[(st * KM + j) * 32]
   bool bounds = false;
   const int n_work = a.T * a.slices;  // < 2^31: slices > 1 only for few rows
   for (unsigned wk = blockIdx.x * kFaninWarps + warp; wk < (unsigned)n_work; wk += gridDim.x * kFaninWarps) {
@@ -258,21 +294,33 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
       tab[lane] = e;
     }
     __syncwarp();
-    uint8_t *orow = a.out + (size_t)t * a.rb_out;
-    for (int v = vbeg + lane; v < vend; v += 32) {
-      uint4 d[KM];
+    auto issue = [&](int v, int st) {
 #pragma unroll
       for (int j = 0; j < KM; ++j)
-        if (vmask >> j & 1u) d[j] = ld_stream_v4((const uint8_t *)read_entry(tab + j).addr + (size_t)v * 16);
+        if (vmask >> j & 1u)
+          cp_async16(stage + (st * KM + j) * 32, (const uint8_t *)read_entry(tab + j).addr + (size_t)v * 16);
+      cp_async_commit();
+    };
+    uint8_t *orow = a.out + (size_t)t * a.rb_out;
+    int st = 0;
+    if (vbeg + lane < vend) issue(vbeg + lane, 0);
+    for (int v = vbeg + lane; v < vend; v += 32, st ^= 1) {
+      if (v + 32 < vend) {
+        issue(v + 32, st ^ 1);
+        cp_async_wait<1>();  // this vector's group is in
+      } else {
+        cp_async_wait<0>();
+      }
       float acc_g[VE], acc_o[VE];
 #pragma unroll
       for (int e = 0; e < VE; ++e) acc_g[e] = acc_o[e] = 0.0f;
 #pragma unroll
       for (int j = 0; j < KM; ++j) {
         if (vmask >> j & 1u) {
+          const uint4 d = stage[(st * KM + j) * 32];
           const float c = read_entry(tab + j).coef;
 #pragma unroll
-          for (int e = 0; e < VE; ++e) acc_g[e] = fmaf(c, Elem<Tin>::get(d[j], e), acc_g[e]);
+          for (int e = 0; e < VE; ++e) acc_g[e] = fmaf(c, Elem<Tin>::get(d, e), acc_g[e]);
         }
         if (lastmask >> j & 1u) {
 #pragma unroll
@@ -296,7 +344,11 @@ __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
 template <typename Tin, typename Tout, int KM>
 cudaError_t launch_two_hop3(const TwoHopArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   const long blocks = ((long)a.T * a.slices + kFaninWarps - 1) / kFaninWarps;  // uncapped, as in pack
-  two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
+  constexpr int smem = kFaninWarps * 2 * KM * 32 * 16;  // two stages of 16-byte slots per lane and row
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t err = set_smem_limit_once(two_hop_fanin_kernel<Tin, Tout, KM>, smem, smem_set);
+  if (err != cudaSuccess) return err;
+  two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, smem, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
 
@@ -322,7 +374,11 @@ cudaError_t launch3(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   const long blocks = (a.n_items >= 0) ? ((long)a.n_items * a.slices + kFaninWarps - 1) / kFaninWarps
                                        : (long)ctx.num_sms * 8;
   if (blocks <= 0) return cudaSuccess;
-  fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, 0, s>>>(a, ctx);
+  constexpr int smem = kFaninWarps * 2 * KM * 32 * 16;  // two stages of 16-byte slots per lane and row
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t err = set_smem_limit_once(fanin_kernel<Tin, Tout, KM>, smem, smem_set);
+  if (err != cudaSuccess) return err;
+  fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, smem, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
 
