@@ -23,6 +23,7 @@ struct PerDevice {
   std::atomic<int *> status{nullptr};
   int *status_out = nullptr;
   int num_sms = 0;
+  int smem_per_sm = 0;
 };
 PerDevice g_dev[kMaxDevices];
 std::mutex g_init_mu;
@@ -40,19 +41,23 @@ int get_ctx(moe::DeviceCtx *ctx) {
     st = d.status.load(std::memory_order_relaxed);
     if (!st) {
       void *p = nullptr, *q = nullptr;
-      int sms = 0;
+      int sms = 0, smem = 0;
       if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return MOE_ERR_CUDA;
       if (cudaGetSymbolAddress(&q, g_status_out) != cudaSuccess) return MOE_ERR_CUDA;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return MOE_ERR_CUDA;
+      if (cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
+        return MOE_ERR_CUDA;
       d.status_out = static_cast<int *>(q);
       d.num_sms = sms;
+      d.smem_per_sm = smem;
       st = static_cast<int *>(p);
       d.status.store(st, std::memory_order_release);
     }
   }
   ctx->status = st;
   ctx->num_sms = d.num_sms;
+  ctx->smem_per_sm = d.smem_per_sm;
   ctx->wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   ctx->silent_tile = g_silent_tile.load(std::memory_order_relaxed);
   return MOE_OK;

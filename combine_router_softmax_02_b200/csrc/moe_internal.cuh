@@ -24,8 +24,9 @@ constexpr int kMaxSlots = 32768;
 struct DeviceCtx {
   int *status;            // per-device status word (first error wins)
   uint64_t wait_limit_ns; // limit of every bounded wait
-  int silent_tile;        // layout scan tile that does not publish (-1: none)
+  int silent_tile;        // layout block that never arrives at its barrier (-1: none)
   int num_sms;
+  int smem_per_sm;        // shared memory per SM, bytes
 };
 
 // ---------------------------------------------------------------- device ----

@@ -47,8 +47,18 @@ struct FanoutArgs {
 // segment advance as one window.  Capping it at 16 blocks per SM with a
 // grid-stride loop split the resident tokens into disjoint windows and cost
 // 2.5% on the 65536-token workload (a write probe shows the same: a sliding
-// window of stores runs at 7.1 TB/s, scattered windows at 6.2-6.9).
+// window of stores runs at 7.1 TB/s, scattered windows at 6.2-6.9); a
+// persistent grid of 2 blocks per SM cost 11%.
+//
+// Residency: fewer concurrent warps write fewer rows at a time, and the DRAM
+// then serves the writes faster.  A large launch (more than 8 blocks per SM;
+// a decode-sized one keeps every warp for latency) therefore reserves just over
+// a third of the SM's shared memory per block (unused), which holds it at 2
+// resident blocks per SM: 5 -> 2 blocks per SM took the 65536-token pack from
+// 1326 to 1302 us and the two-hop pack from 555 to 548 us (3 and 4 blocks per
+// SM fell in between, 1 block was slower on the first).
 constexpr int kU = 2;
+constexpr int kResidentBlocks = 2;
 
 template <int KM, int NL, int U>
 __global__ void __launch_bounds__(256) fanout_kernel(FanoutArgs a, DeviceCtx ctx) {
@@ -101,7 +111,14 @@ template <int KM, int NL>
 cudaError_t launch_kn(const FanoutArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   const int wpb = 8;
   const long blocks = ((long)a.n_items * a.slices + wpb - 1) / wpb;
-  fanout_kernel<KM, NL, kU><<<(unsigned)blocks, wpb * 32, 0, s>>>(a, ctx);
+  int smem = 0;
+  if (blocks > 8L * ctx.num_sms && ctx.smem_per_sm > 0) {  // large launches only (decode keeps all warps)
+    smem = ctx.smem_per_sm / (kResidentBlocks + 1) + 1024;  // room for 2 blocks, not for 3
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t err = set_smem_limit_once(fanout_kernel<KM, NL, kU>, 160 * 1024, smem_set);
+    if (err != cudaSuccess) return err;
+  }
+  fanout_kernel<KM, NL, kU><<<(unsigned)blocks, wpb * 32, smem, s>>>(a, ctx);
   return count_launch(cudaGetLastError());
 }
 
