@@ -12,6 +12,6 @@ from ._binding import (BF16, DEDUP, F16, F32, MOE_OK, PER_PICK, STATUS_NAMES, TW
                        Layout, MoeError, build_layout, check_status, combine, debug_set_wait,
                        demand_hist, get_status, kernel_launches, layout_workspace_size, lib, moe_layout, pack,
                        replica_assign, route_topk, status_string, dispatch_stats,
-                       token_balanced_assign, STAT_NAMES, route_layout_single_replica,
+                       token_balanced_assign, STAT_NAMES, route_layout_single_replica, route_assign_layout,
                        coselection_hist, correlated_placement)
 from .path import DispatchCombine, HostPipeline  # noqa: F401

@@ -66,6 +66,9 @@ _SIGS = {
     "moe_route_layout_single_replica": (ctypes.c_int, [_P, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _I,
                                                        _P, _P, _P, _P, ctypes.POINTER(moe_layout),
                                                        _P, _SZ, _S]),
+    "moe_route_assign_layout": (ctypes.c_int, [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _I, _I,
+                                               _I, _I, _P, _P, _P, _P, _P, _P,
+                                               ctypes.POINTER(moe_layout), _P, _SZ, _S]),
     "moe_coselection_hist": (ctypes.c_int, [_P, _I, _I, _I, _P, _S]),
     "moe_correlated_placement": (ctypes.c_int, [_P, _P, _I, _I, _P, _S]),
     "moe_dispatch_stats": (ctypes.c_int, [_P, _I, _P, _I, _P, _S]),
@@ -368,6 +371,38 @@ def route_layout_single_replica(logits: torch.Tensor, k: int, expert_rank: torch
         _p(rank_active), ctypes.byref(L.struct), _p(L.workspace), L.workspace.numel(), _stream(stream)),
         "moe_route_layout_single_replica")
     return topk_idx, topk_w, counts
+
+
+def route_assign_layout(logits: torch.Tensor, k: int, replica_offsets, replica_slots, slot_rank,
+                        layout: Layout, n_groups: int = 0, groups_per_token: int = 0,
+                        renormalize: bool = False, topk_idx=None, topk_w=None, counts=None,
+                        expert_slot=None, expert_rank=None, rank_active=None, stream=None):
+    """route_topk + demand_hist + replica_assign + build_layout in one launch, for
+    any replica map.  Returns (topk_idx, topk_w, counts, expert_slot, expert_rank,
+    rank_active)."""
+    _need(logits, torch.float32, "logits", 2)
+    for t, n in ((replica_offsets, "replica_offsets"), (replica_slots, "replica_slots"),
+                 (slot_rank, "slot_rank")):
+        _need(t, torch.int32, n, 1)
+    T, E = logits.shape
+    L = layout
+    if (T, k, E) != (L.T, L.k, L.E):
+        raise ValueError("logits / k do not match the layout's sizes")
+    dev = logits.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    topk_idx = torch.empty((T, k), **i32) if topk_idx is None else topk_idx
+    topk_w = torch.empty((T, k), dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    counts = torch.empty(E, **i32) if counts is None else counts
+    expert_slot = torch.empty(E, **i32) if expert_slot is None else expert_slot
+    expert_rank = torch.empty(E, **i32) if expert_rank is None else expert_rank
+    rank_active = torch.empty(L.R, **i32) if rank_active is None else rank_active
+    _check(lib().moe_route_assign_layout(
+        _p(logits), T, E, k, n_groups, groups_per_token, int(renormalize), _p(replica_offsets),
+        _p(replica_slots), replica_slots.numel(), _p(slot_rank), slot_rank.numel(), L.tokens_per_rank,
+        L.R, L.ranks_per_group, L.mode, _p(topk_idx), _p(topk_w), _p(counts), _p(expert_slot),
+        _p(expert_rank), _p(rank_active), ctypes.byref(L.struct), _p(L.workspace), L.workspace.numel(),
+        _stream(stream)), "moe_route_assign_layout")
+    return topk_idx, topk_w, counts, expert_slot, expert_rank, rank_active
 
 
 def coselection_hist(topk_idx: torch.Tensor, E: int, cosel=None, stream=None):

@@ -30,29 +30,9 @@ __global__ void __launch_bounds__(kTile) layout_kernel(LayoutArgs a, DeviceCtx c
   int *sm = reinterpret_cast<int *>(smem_raw);
   __shared__ int s_flag;
   const SmemPlan P = smem_plan(a.E, a.NBp, a.R, false);
-  const int lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * a.chunk, t1 = min(a.T, t0 + a.chunk);
   smem_init(a, P, sm);
-
-  // phase 1: the block's rows per bin (a one-tile chunk keeps its picks,
-  // weights included, and its ballots for phase 2)
-  const bool one_tile = t1 - t0 <= kTile;
-  bool bad = false;
-  int c[4] = {0, 0, 0, 0};
-  TokenPicks<KM> p;
-  Ballots bl{0u, 0u, 0u, 0u};
-  for (int base = t0; base < t1; base += kTile) {
-    const int t = base + (int)threadIdx.x;
-    load_picks<KM, MODE>(a, sm + P.er, t, t < t1, one_tile, p, bad);
-    count_tile<KM, MODE>(a, p, t < t1, lane, sm + P.cnt, c, bl);
-  }
-  flush_counts<MODE>(a, lane, sm + P.cnt, c);
-  if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
-  publish_counts(a, P, sm);
-  if (!grid_barrier(a, ctx, &s_flag)) return;
-
-  // phase 2: offsets and rows
-  phase2<KM, MODE>(a, P, sm, t0, t1, ctx, one_tile ? &p : nullptr, one_tile ? &bl : nullptr);
+  layout_phases<KM, MODE>(a, P, sm, t0, t1, ctx, &s_flag, 1);
 }
 
 std::atomic<unsigned long long> g_smem_set[4][3];
@@ -68,7 +48,7 @@ cudaError_t launch_k(const LayoutArgs &a0, int kind, const DeviceCtx &ctx, cudaS
   if ((err = max_resident_blocks((const void *)kern, smem, ctx, resident)) != cudaSuccess) return err;
   split_tokens(a.T, resident < kBlocksPerSm * ctx.num_sms ? resident : kBlocksPerSm * ctx.num_sms,
                a.nblk, a.chunk);
-  if ((err = cudaMemsetAsync(a.bar, 0, sizeof(int) * kHeaderInts, s)) != cudaSuccess) return err;
+  if ((err = cudaMemsetAsync(a.bar, 0, sizeof(int) * 16, s)) != cudaSuccess) return err;
   void *args[] = {&a, const_cast<DeviceCtx *>(&ctx)};
   err = cudaLaunchCooperativeKernel((const void *)kern, dim3(a.nblk), dim3(kTile), args, smem, s);
   if (err != cudaSuccess) return err;
@@ -104,6 +84,7 @@ LayoutArgs make_layout_args(const int *idx, const float *w, const int *expert_ra
   a.nblk = 0;
   a.chunk = 0;
   a.bar = static_cast<unsigned *>(ws);
+  a.cnt = static_cast<int *>(ws) + 16;
   a.agg = static_cast<int *>(ws) + kHeaderInts;
   a.L = L;
   return a;
@@ -135,7 +116,7 @@ cudaError_t max_resident_blocks(const void *kernel, size_t smem, const DeviceCtx
 size_t layout_workspace_bytes(int T, int k, int E, int R, int rpg, int mode) {
   (void)k;
   const int NBp = (layout::num_bins(E, R, rpg, mode) + 3) & ~3;
-  long rows = ((long)T + 31) / 32;  // chunks are multiples of 32 tokens
+  long rows = ((long)T + 7) / 8;  // chunks are multiples of 8 tokens
   if (rows > layout::kMaxBlocks) rows = layout::kMaxBlocks;
   if (rows < 1) rows = 1;
   return sizeof(int) * (layout::kHeaderInts + (size_t)rows * NBp);

@@ -26,7 +26,7 @@ constexpr int kWarps = kTile / 32;
 constexpr int kMaxBins = kMaxE;  // >= max(E, R + G)
 constexpr int kMaxBlocks = 512;  // grid cap (rows of the count table)
 constexpr int kBlocksPerSm = 2;  // layout grid: blocks per SM (when resident)
-constexpr int kHeaderInts = 16;  // barrier words at the start of the workspace
+constexpr int kHeaderInts = 16 + kMaxE;  // workspace header: barrier words, then a demand scratch
 constexpr unsigned kFull = 0xffffffffu;
 
 struct LayoutArgs {
@@ -35,8 +35,9 @@ struct LayoutArgs {
   const int *expert_rank;
   int T, tpr, k, E, R, rpg, G, mode, NB, NBp;
   int nblk;        // blocks of the launch
-  int chunk;       // tokens per block, a multiple of 32
+  int chunk;       // tokens per block, a multiple of 8
   unsigned *bar;   // [0] barrier arrivals, [1] blocks done
+  int *cnt;        // [E] demand scratch of the fused front ends (cleared with the barrier words)
   int *agg;        // [nblk][NBp] per-block bin counts
   moe_layout L;
 };
@@ -252,21 +253,24 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
 }
 
 // Grid-wide barrier over the launch's blocks (all resident: cooperative
-// launch).  Returns false on every thread of the block when the wait ran out
-// (MOE_ERR_TIMEOUT is set) or the block is the test hook's silent block, which
-// never arrives.
-__device__ __forceinline__ bool grid_barrier(const LayoutArgs &a, const DeviceCtx &ctx, int *s_flag) {
+// launch); `round` counts the barriers of the launch from 1 (each block adds
+// one arrival per round).  Returns false on every thread of the block when the
+// wait ran out (MOE_ERR_TIMEOUT is set) or the block is the test hook's silent
+// block, which never arrives.
+__device__ __forceinline__ bool grid_barrier(const LayoutArgs &a, const DeviceCtx &ctx, int *s_flag,
+                                             unsigned round = 1) {
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
+    const unsigned target = round * (unsigned)a.nblk;
     if ((int)blockIdx.x == ctx.silent_tile) {
       ok = 0;
     } else {
       red_release_add(a.bar, 1u);
-      if (ld_acquire_u32(a.bar) < (unsigned)a.nblk) {
+      if (ld_acquire_u32(a.bar) < target) {
         const uint64_t t0 = global_ns();
-        while (ld_acquire_u32(a.bar) < (unsigned)a.nblk) {
+        while (ld_acquire_u32(a.bar) < target) {
           __nanosleep(32);
           if (global_ns() - t0 > ctx.wait_limit_ns || ld_volatile_i32(ctx.status) == MOE_ERR_TIMEOUT) {
             set_status(ctx.status, MOE_ERR_TIMEOUT);
@@ -602,10 +606,36 @@ __device__ __forceinline__ void publish_counts(const LayoutArgs &a, const SmemPl
 
 // Clears the block's shared counters and loads the expert -> rank map.
 __device__ __forceinline__ void smem_init(const LayoutArgs &a, const SmemPlan &P, int *sm) {
-  for (int i = threadIdx.x; i < a.E; i += kTile) sm[P.er + i] = a.expert_rank[i];
+  for (int i = threadIdx.x; i < a.E; i += kTile) sm[P.er + i] = __ldcg(a.expert_rank + i);
   for (int i = threadIdx.x; i < a.NBp; i += kTile) sm[P.cnt + i] = 0;
   for (int i = threadIdx.x; i < a.R * a.R; i += kTile) sm[P.send + i] = 0;
   __syncthreads();
+}
+
+// Both layout phases over the block's chunk [t0, t1), after smem_init: phase
+// 1 counts the chunk's rows per bin (a one-tile chunk keeps its picks and
+// ballots), the grid barrier `round` publishes the count table, phase 2
+// writes the rows.  Returns false when the barrier gave up.
+template <int KM, int MODE>
+__device__ __forceinline__ bool layout_phases(const LayoutArgs &a, const SmemPlan &P, int *sm, int t0,
+                                              int t1, DeviceCtx ctx, int *s_flag, unsigned round) {
+  const int lane = threadIdx.x & 31;
+  const bool one_tile = t1 - t0 <= kTile;
+  bool bad = false;
+  int c[4] = {0, 0, 0, 0};
+  TokenPicks<KM> p;
+  Ballots bl{0u, 0u, 0u, 0u};
+  for (int base = t0; base < t1; base += kTile) {
+    const int t = base + (int)threadIdx.x;
+    load_picks<KM, MODE>(a, sm + P.er, t, t < t1, one_tile, p, bad);
+    count_tile<KM, MODE>(a, p, t < t1, lane, sm + P.cnt, c, bl);
+  }
+  flush_counts<MODE>(a, lane, sm + P.cnt, c);
+  if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
+  publish_counts(a, P, sm);
+  if (!grid_barrier(a, ctx, s_flag, round)) return false;
+  phase2<KM, MODE>(a, P, sm, t0, t1, ctx, one_tile ? &p : nullptr, one_tile ? &bl : nullptr);
+  return true;
 }
 
 // ---------------------------------------------------------------- host ----
@@ -618,12 +648,14 @@ inline int num_bins(int E, int R, int rpg, int mode) {
 inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 // Blocks and chunk of a launch: at most `max_blocks` blocks, chunks of a
-// multiple of 32 tokens.
-inline void split_tokens(int T, int max_blocks, int &nblk, int &chunk) {
+// multiple of `granule` tokens (32 for the layout kernel, a thread per token;
+// 8 for the fused front ends, whose routing phase gives each warp a token).
+// The workspace holds a count-table row per 8 tokens, up to kMaxBlocks.
+inline void split_tokens(int T, int max_blocks, int &nblk, int &chunk, int granule = 32) {
   if (max_blocks < 1) max_blocks = 1;
   if (max_blocks > kMaxBlocks) max_blocks = kMaxBlocks;
   chunk = (int)(((long)T + max_blocks - 1) / max_blocks);
-  chunk = (chunk + 31) & ~31;
+  chunk = (chunk + granule - 1) / granule * granule;
   nblk = (int)(((long)T + chunk - 1) / chunk);
 }
 

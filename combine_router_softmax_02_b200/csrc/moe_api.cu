@@ -292,16 +292,18 @@ int moe_token_balanced_assign(const int32_t *counts, int32_t E, const int32_t *r
 
 }  // extern "C"
 
-extern "C" int moe_route_layout_single_replica(
-    const float *logits, int32_t T, int32_t E, int32_t k, int32_t n_groups,
-    int32_t groups_per_token, int32_t renormalize, const int32_t *expert_rank,
-    int32_t tokens_per_rank, int32_t R, int32_t ranks_per_group, int32_t mode, int32_t *topk_idx,
-    float *topk_w, int32_t *counts, int32_t *rank_active, moe_layout *layout, void *workspace,
-    size_t workspace_bytes, moe_stream_t stream) {
-  // the checks of moe_route_topk and moe_build_layout, launch-free
+namespace {
+
+// The checks of moe_route_topk and moe_build_layout for the fused front ends
+// (launch-free).
+int check_front(const float *logits, int32_t T, int32_t E, int32_t k, int32_t n_groups,
+                int32_t groups_per_token, int32_t renormalize, int32_t tokens_per_rank, int32_t R,
+                int32_t ranks_per_group, int32_t mode, const int32_t *topk_idx, const float *topk_w,
+                const int32_t *counts, const moe_layout *layout, const void *workspace,
+                size_t workspace_bytes) {
   if (!layout || T < 0 || !valid_ekr(E, k) || R < 1 || R > moe::kMaxR) return MOE_ERR_INVALID_ARG;
   if ((int64_t)T * k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
-  if (!counts || !expert_rank) return MOE_ERR_INVALID_ARG;
+  if (!counts) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
   if (renormalize != 0 && renormalize != 1) return MOE_ERR_INVALID_ARG;
   if (n_groups != 0 || groups_per_token != 0) {
@@ -313,7 +315,7 @@ extern "C" int moe_route_layout_single_replica(
   if (tokens_per_rank < 1 || (int64_t)tokens_per_rank * R < T) return MOE_ERR_INVALID_ARG;
   if (mode == MOE_LAYOUT_TWO_HOP && (ranks_per_group < 1 || ranks_per_group > R || R % ranks_per_group))
     return MOE_ERR_INVALID_ARG;
-  moe_layout &L = *layout;
+  const moe_layout &L = *layout;
   if (!L.rank_offsets || !L.send_counts || !L.num_rows || L.capacity < 0) return MOE_ERR_INVALID_ARG;
   if (T > 0 && !L.token_rows) return MOE_ERR_INVALID_ARG;
   if (L.capacity > 0 && (!L.row_token || !L.row_coef)) return MOE_ERR_INVALID_ARG;
@@ -325,18 +327,71 @@ extern "C" int moe_route_layout_single_replica(
   }
   const size_t need = moe::layout_workspace_bytes(T, k, E, R, ranks_per_group, mode);
   if (T > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return MOE_ERR_INVALID_ARG;
-  moe::DeviceCtx ctx;
-  int rc = get_ctx(&ctx);
-  if (rc) return rc;
+  return MOE_OK;
+}
+
+void fill_layout_shape(moe_layout &L, int32_t T, int32_t k, int32_t E, int32_t R,
+                       int32_t ranks_per_group, int32_t mode) {
   L.T = T;
   L.k = k;
   L.R = R;
   L.E = E;
   L.ranks_per_group = (mode == MOE_LAYOUT_TWO_HOP) ? ranks_per_group : 1;
   L.mode = mode;
+}
+
+}  // namespace
+
+extern "C" int moe_route_layout_single_replica(
+    const float *logits, int32_t T, int32_t E, int32_t k, int32_t n_groups,
+    int32_t groups_per_token, int32_t renormalize, const int32_t *expert_rank,
+    int32_t tokens_per_rank, int32_t R, int32_t ranks_per_group, int32_t mode, int32_t *topk_idx,
+    float *topk_w, int32_t *counts, int32_t *rank_active, moe_layout *layout, void *workspace,
+    size_t workspace_bytes, moe_stream_t stream) {
+  int rc = check_front(logits, T, E, k, n_groups, groups_per_token, renormalize, tokens_per_rank, R,
+                       ranks_per_group, mode, topk_idx, topk_w, counts, layout, workspace,
+                       workspace_bytes);
+  if (rc) return rc;
+  if (!expert_rank) return MOE_ERR_INVALID_ARG;
+  moe::DeviceCtx ctx;
+  rc = get_ctx(&ctx);
+  if (rc) return rc;
+  moe_layout &L = *layout;
+  fill_layout_shape(L, T, k, E, R, ranks_per_group, mode);
   return launched(moe::launch_route_layout_static(
       logits, T, E, k, n_groups, groups_per_token, renormalize, expert_rank, tokens_per_rank, R,
       ranks_per_group, mode, topk_idx, topk_w, counts, rank_active, L, workspace, ctx,
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+extern "C" int moe_route_assign_layout(
+    const float *logits, int32_t T, int32_t E, int32_t k, int32_t n_groups, int32_t groups_per_token,
+    int32_t renormalize, const int32_t *replica_offsets, const int32_t *replica_slots,
+    int32_t n_replica_entries, const int32_t *slot_rank, int32_t S, int32_t tokens_per_rank, int32_t R,
+    int32_t ranks_per_group, int32_t mode, int32_t *topk_idx, float *topk_w, int32_t *counts,
+    int32_t *expert_slot, int32_t *expert_rank, int32_t *rank_active, moe_layout *layout,
+    void *workspace, size_t workspace_bytes, moe_stream_t stream) {
+  int rc = check_front(logits, T, E, k, n_groups, groups_per_token, renormalize, tokens_per_rank, R,
+                       ranks_per_group, mode, topk_idx, topk_w, counts, layout, workspace,
+                       workspace_bytes);
+  if (rc) return rc;
+  // the checks of moe_replica_assign
+  if (S < 1 || S > moe::kMaxSlots || n_replica_entries < 0 || n_replica_entries > moe::kMaxSlots)
+    return MOE_ERR_INVALID_ARG;
+  if (!replica_offsets || !slot_rank || !expert_slot || !expert_rank || !rank_active)
+    return MOE_ERR_INVALID_ARG;
+  if (n_replica_entries > 0 && !replica_slots) return MOE_ERR_INVALID_ARG;
+  if (moe::front_smem_bytes(E, k, R, ranks_per_group, mode, n_replica_entries) > (size_t)moe::kFrontSmemMax)
+    return MOE_ERR_UNSUPPORTED;
+  moe::DeviceCtx ctx;
+  rc = get_ctx(&ctx);
+  if (rc) return rc;
+  moe_layout &L = *layout;
+  fill_layout_shape(L, T, k, E, R, ranks_per_group, mode);
+  return launched(moe::launch_route_assign_layout(
+      logits, T, E, k, n_groups, groups_per_token, renormalize, replica_offsets, replica_slots,
+      n_replica_entries, slot_rank, S, tokens_per_rank, R, ranks_per_group, mode, topk_idx, topk_w,
+      counts, expert_slot, expert_rank, rank_active, L, workspace, ctx,
       reinterpret_cast<cudaStream_t>(stream)));
 }
 

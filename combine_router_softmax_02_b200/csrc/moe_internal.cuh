@@ -134,6 +134,17 @@ cudaError_t launch_route_layout_static(const float *logits, int T, int E, int k,
                                        float *w, int *counts, int *rank_active,
                                        const moe_layout &L, void *ws, const DeviceCtx &ctx,
                                        cudaStream_t s);
+// The single-launch front end for any replica map (route_assign_layout.cu):
+// shared memory it needs for these sizes, and the largest it may take.
+constexpr int kFrontSmemMax = 200 * 1024;
+size_t front_smem_bytes(int E, int k, int R, int rpg, int mode, int n_entries);
+cudaError_t launch_route_assign_layout(const float *logits, int T, int E, int k, int n_groups, int gpt,
+                                       int renorm, const int *off, const int *slots, int n_entries,
+                                       const int *slot_rank, int S, int tokens_per_rank, int R,
+                                       int rpg, int mode, int *idx, float *w, int *counts,
+                                       int *expert_slot, int *expert_rank, int *rank_active,
+                                       const moe_layout &L, void *ws, const DeviceCtx &ctx,
+                                       cudaStream_t s);
 cudaError_t launch_coselection(const int *idx, int T, int k, int E, int *C, const DeviceCtx &ctx,
                                cudaStream_t s);
 cudaError_t launch_placement(const int *C, const int *counts, int E, int R, int *expert_rank,

@@ -125,8 +125,8 @@ cudaError_t launch_fused(const RouteArgs &ra0, const LayoutArgs &a0, int slot, c
   int resident = 0;
   if ((err = layout::max_resident_blocks((const void *)kern, smem, ctx, resident)) != cudaSuccess)
     return err;
-  layout::split_tokens(a.T, resident, a.nblk, a.chunk);
-  if ((err = cudaMemsetAsync(a.bar, 0, sizeof(int) * layout::kHeaderInts, s)) != cudaSuccess) return err;
+  layout::split_tokens(a.T, resident, a.nblk, a.chunk, 8);
+  if ((err = cudaMemsetAsync(a.bar, 0, sizeof(int) * 16, s)) != cudaSuccess) return err;
   void *args[] = {&ra, &a, const_cast<DeviceCtx *>(&ctx)};
   err = cudaLaunchCooperativeKernel((const void *)kern, dim3(a.nblk), dim3(kTile), args, smem, s);
   if (err != cudaSuccess) return err;

@@ -60,6 +60,13 @@ class DispatchCombine:
                                       self.groups_per_token, self.renormalize, self.topk_idx,
                                       self.topk_w, self.counts, self.rank_active)
 
+    def route_one_launch(self, logits: torch.Tensor):
+        """The same outputs as route(), from one launch (moe_route_assign_layout)."""
+        B.route_assign_layout(logits, self.k, self.replica_offsets, self.replica_slots, self.slot_rank,
+                              self.layout, self.n_groups, self.groups_per_token, self.renormalize,
+                              self.topk_idx, self.topk_w, self.counts, self.expert_slot,
+                              self.expert_rank, self.rank_active)
+
     def dispatch(self, logits: torch.Tensor, x: torch.Tensor) -> torch.Tensor:
         self.route(logits)
         B.pack(x, self.layout, self.packed, self.packed_hop1)

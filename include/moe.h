@@ -203,7 +203,7 @@ MOE_API int moe_build_layout(const int32_t *topk_idx, const float *topk_w, const
  * Returns MOE_ERR_UNSUPPORTED, before anything is launched, when
  * moe_layout_workspace_size() for these sizes exceeds
  * MOE_LAYOUT_STATIC_SCRATCH_BYTES (for example 65536 tokens over 64 ranks
- * needs 131 KB in DEDUP mode).  The first call on a device looks up the
+ * needs 135 KB in DEDUP mode).  The first call on a device looks up the
  * array's device address with that device current; make that first call
  * before any stream capture.  All calls share the one array, whose contents
  * persist from call to call (each call clears what must start at zero):
@@ -277,6 +277,29 @@ MOE_API int moe_route_layout_single_replica(
     int32_t tokens_per_rank, int32_t R, int32_t ranks_per_group, int32_t mode, int32_t *topk_idx,
     float *topk_w, int32_t *counts, int32_t *rank_active, moe_layout *layout, void *workspace,
     size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * moe_route_topk, moe_demand_hist, moe_replica_assign and moe_build_layout in
+ * one launch, for any replica map.  Source: "METRO AllGather vs AllToAll for
+ * MoE decode", section "changes the routing information" (every rank computes
+ * the global routing, the demand vector and the assignment: at decode sizes
+ * their launch cost is what the global information costs).  One cooperative
+ * kernel routes the tokens and counts the demand vector, one block runs the
+ * METRO greedy over it, and every block then builds its part of the layout,
+ * with grid barriers between the phases.  Every output equals that of the four
+ * separate calls.  Arguments as in those calls; the workspace is
+ * moe_layout_workspace_size() bytes as for moe_build_layout.  Returns
+ * MOE_ERR_UNSUPPORTED, before anything is launched, if one block's shared
+ * memory cannot hold the replica map and the layout bins (within the limits of
+ * moe_replica_assign and moe_build_layout they take at most 139 KB).
+ */
+MOE_API int moe_route_assign_layout(
+    const float *logits, int32_t T, int32_t E, int32_t k, int32_t n_groups, int32_t groups_per_token,
+    int32_t renormalize, const int32_t *replica_offsets, const int32_t *replica_slots,
+    int32_t n_replica_entries, const int32_t *slot_rank, int32_t S, int32_t tokens_per_rank, int32_t R,
+    int32_t ranks_per_group, int32_t mode, int32_t *topk_idx, float *topk_w, int32_t *counts,
+    int32_t *expert_slot, int32_t *expert_rank, int32_t *rank_active, moe_layout *layout,
+    void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /*
  * Co-selection counts: cosel[e*E + f] = number of tokens whose picks include

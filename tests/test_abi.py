@@ -64,12 +64,14 @@ def test_status_strings(lib):
 
 
 def test_workspace_size(lib):
-    # 64 bytes of barrier words, then one int per (block, bin) with bins padded
-    # to a multiple of 4; at most 512 blocks, and at most one per 32 tokens
-    assert moe.layout_workspace_size(65536, 8, 256, 64, 1, moe.DEDUP) == 64 + 512 * 64 * 4
-    assert moe.layout_workspace_size(100, 6, 64, 32, 1, moe.PER_PICK) == 64 + 4 * 64 * 4
-    assert moe.layout_workspace_size(32768, 8, 128, 64, 8, moe.TWO_HOP) == 64 + 512 * 72 * 4
-    assert moe.layout_workspace_size(1, 2, 10, 3, 1, moe.DEDUP) == 64 + 1 * 4 * 4
+    # a header of 16 barrier words and a 1024-entry demand scratch, then one int
+    # per (block, bin) with bins padded to a multiple of 4; at most 512 blocks,
+    # and at most one per 8 tokens
+    H = 4 * (16 + 1024)
+    assert moe.layout_workspace_size(65536, 8, 256, 64, 1, moe.DEDUP) == H + 512 * 64 * 4
+    assert moe.layout_workspace_size(100, 6, 64, 32, 1, moe.PER_PICK) == H + 13 * 64 * 4
+    assert moe.layout_workspace_size(32768, 8, 128, 64, 8, moe.TWO_HOP) == H + 512 * 72 * 4
+    assert moe.layout_workspace_size(1, 2, 10, 3, 1, moe.DEDUP) == H + 1 * 4 * 4
     assert moe.layout_workspace_size(10, 3, 2, 4, 1, moe.DEDUP) == 0        # k > E
     assert moe.layout_workspace_size(10, 2, 8, 65, 1, moe.DEDUP) == 0       # R > 64
     assert moe.layout_workspace_size(10, 2, 8, 8, 3, moe.TWO_HOP) == 0      # rpg does not divide R
