@@ -102,3 +102,44 @@ def test_bad_arguments_rejected_before_launch(lib):
     assert lib.moe_pack(ctypes.c_void_p(8), 1, 8, ctypes.byref(L), P, None, None) == INVALID  # misaligned
     assert lib.moe_combine(P, 1, 8, ctypes.byref(L), None, P, 7, None, None) == INVALID
     assert lib.moe_debug_set_wait(0, -2) == INVALID
+
+
+def test_one_launch_front_ends_reject_bad_arguments(lib):
+    """moe_route_assign_layout and moe_route_layout_single_replica check their
+    arguments on the host and return before any launch (no GPU is touched)."""
+    P = ctypes.c_void_p(256)
+    INVALID, UNSUPPORTED = 1, 2
+    L = moe.moe_layout()
+    L.rank_offsets = L.send_counts = L.num_rows = L.token_rows = L.row_token = L.row_coef = 256
+    L.capacity = 64
+    ws = 1 << 20
+
+    def ral(T=32, E=16, k=2, ng=0, gpt=0, ren=0, n_entries=16, S=16, tpr=8, R=4, rpg=1, mode=1,
+            logits=P, offs=P, slots=P, srank=P, counts=P, eslot=P, erank=P, active=P, wsb=ws, wsp=P):
+        return lib.moe_route_assign_layout(logits, T, E, k, ng, gpt, ren, offs, slots, n_entries, srank, S,
+                                           tpr, R, rpg, mode, P, P, counts, eslot, erank, active,
+                                           ctypes.byref(L), wsp, wsb, None)
+
+    assert ral(k=17) == INVALID                      # k > E
+    assert ral(E=2048) == INVALID                    # E > 1024
+    assert ral(R=65) == INVALID                      # R > 64
+    assert ral(mode=3) == INVALID                    # no such layout mode
+    assert ral(tpr=7) == INVALID                     # tokens_per_rank * R < T
+    assert ral(ng=3, gpt=1) == INVALID               # groups do not divide E
+    assert ral(ren=2) == INVALID                     # renormalize is 0 or 1
+    assert ral(S=0) == INVALID                       # no replica slots
+    assert ral(n_entries=40000) == INVALID           # more replica entries than slots allowed
+    assert ral(offs=None) == INVALID
+    assert ral(slots=None) == INVALID                # entries but no slot list
+    assert ral(srank=None) == INVALID
+    assert ral(counts=None) == INVALID
+    assert ral(eslot=None) == INVALID
+    assert ral(erank=None) == INVALID
+    assert ral(active=None) == INVALID
+    assert ral(logits=None) == INVALID
+    assert ral(wsb=8) == INVALID                     # workspace too small
+    assert ral(wsp=ctypes.c_void_p(264)) == INVALID  # workspace not 16-byte aligned
+    assert ral(mode=2, rpg=3) == INVALID             # ranks per group must divide R
+    assert ral(T=1 << 28, k=16, tpr=1 << 26) == UNSUPPORTED  # T * k overflows 31 bits
+    assert lib.moe_route_layout_single_replica(P, 32, 16, 2, 0, 0, 0, None, 8, 4, 1, 1, P, P, P, P,
+                                               ctypes.byref(L), P, ws, None) == INVALID  # no expert_rank
