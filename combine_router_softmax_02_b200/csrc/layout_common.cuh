@@ -23,7 +23,6 @@ namespace layout {
 
 constexpr int kTile = 256;  // threads per block, tokens per phase-2 tile
 constexpr int kWarps = kTile / 32;
-constexpr int kMaxBins = kMaxE;  // >= max(E, R + G)
 constexpr int kMaxBlocks = 512;  // grid cap (rows of the count table)
 constexpr int kBlocksPerSm = 2;  // layout grid: blocks per SM (when resident)
 constexpr int kHeaderInts = 16 + kMaxE;  // workspace header: barrier words, then a demand scratch
@@ -116,12 +115,6 @@ __device__ __forceinline__ void load_picks(const LayoutArgs &a, const int *s_er,
           p.present &= ~(1u << j);
         }
   }
-}
-
-__device__ __forceinline__ unsigned lanemask_lt() {
-  unsigned m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
 }
 
 __device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
@@ -644,8 +637,6 @@ inline int num_bins(int E, int R, int rpg, int mode) {
   if (mode == MOE_LAYOUT_TWO_HOP) return R + R / rpg;
   return R;
 }
-
-inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 // Blocks and chunk of a launch: at most `max_blocks` blocks, chunks of a
 // multiple of `granule` tokens (32 for the layout kernel, a thread per token;

@@ -51,12 +51,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ unsigned lanes_below() {
-  unsigned m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
 // Per-lane constants of a routing warp.  FULL: E == 32 * EPL, every slot
 // holds an expert.
 template <int EPL, bool FULL>
@@ -154,7 +148,7 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
   }
 
   // compaction in ascending expert order: slot j of lane l is expert l + 32 j
-  const unsigned below = lanes_below();
+  const unsigned below = lanemask_lt();
   unsigned total = 0;
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
