@@ -13,30 +13,44 @@
 namespace moe {
 namespace {
 
+constexpr int kPer = 8;  // picks per thread per pass, all loaded before any is counted
+
 __global__ void __launch_bounds__(256) demand_hist_kernel(const int *__restrict__ idx, long n,
                                                           int E, int *__restrict__ counts,
                                                           DeviceCtx ctx) {
   extern __shared__ int h[];
   for (int i = threadIdx.x; i < E; i += blockDim.x) h[i] = 0;
   __syncthreads();
-  const long stride = (long)gridDim.x * blockDim.x;
-  // every lane of a warp runs the same number of iterations, so the warp is
-  // converged at match.any
-  const long base0 = (long)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  // a pass covers kPer warp-widths per warp: lane l of warp w takes picks
+  // base + j * 32 + l, j < kPer (coalesced per j); every lane of a warp runs
+  // the same passes, so the warp is converged at match.any
+  const long per_block = (long)blockDim.x * kPer;
+  const long stride = (long)gridDim.x * per_block;
   const int lane = threadIdx.x & 31;
+  const long base0 = (long)blockIdx.x * per_block + (long)(threadIdx.x >> 5) * 32 * kPer;
   bool bad = false;
   for (long base = base0; base < n; base += stride) {
-    const long i = base + lane;
-    int e = -1;
-    if (i < n) {
-      e = __ldcs(idx + i);
-      if ((unsigned)e >= (unsigned)E) {
-        bad = true;
-        e = -1;
+    int e[kPer];
+    unsigned live = 0;  // which of this lane's slots hold a pick
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const long i = base + j * 32 + lane;
+      e[j] = 0;
+      if (i < n) {
+        e[j] = __ldcs(idx + i);
+        live |= 1u << j;
       }
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&h[e], __popc(peers));
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      int v = (live >> j & 1u) ? e[j] : -1;
+      if ((live >> j & 1u) && (unsigned)v >= (unsigned)E) {
+        bad = true;
+        v = -1;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, v);
+      if (v >= 0 && lane == __ffs(peers) - 1) atomicAdd(&h[v], __popc(peers));
+    }
   }
   if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
   __syncthreads();
@@ -52,7 +66,7 @@ cudaError_t launch_demand_hist(const int *idx, int T, int k, int E, int *counts,
   if (err != cudaSuccess) return err;
   const long n = (long)T * k;
   if (n == 0) return cudaSuccess;
-  long blocks = (n + 256 * 8 - 1) / (256 * 8);
+  long blocks = (n + 256 * kPer - 1) / (256 * kPer);
   const long cap = (long)ctx.num_sms * 2;
   if (blocks > cap) blocks = cap;
   demand_hist_kernel<<<(unsigned)blocks, 256, sizeof(int) * (size_t)E, s>>>(idx, n, E, counts, ctx);

@@ -89,6 +89,11 @@ def test_hist_bad_id_and_skew(moe):
     assert moe.get_status() == 6
     c = c_d.cpu().numpy()
     assert c[0] == 5000 and c[2] == 4999 and c.sum() == 5000 * 4 - 1
+    idx[17, 2] = 2
+    idx[4999, 3] = -1                             # negative, in the ragged last pass
+    c = moe.demand_hist(to_dev(idx), 8).cpu().numpy()
+    assert moe.get_status() == 6
+    assert c[3] == 4999 and c.sum() == 5000 * 4 - 1
 
 
 def _assign_dev(moe, counts, rm_off, rm_slots, slot_rank, R):
