@@ -35,6 +35,11 @@ def test_route_full_size_configs(moe, name):
     (700, 128, 8, 8, 4, 0, False),      # group-limited, the two-hop config's shape
     (300, 96, 5, 32, 3, 0, True),       # 32 groups of 3, ties
     (129, 32, 4, 4, 1, 0, True),
+    (257, 256, 8, 4, 2, 0, True),       # groups of 64: two whole slots each
+    (257, 256, 8, 8, 3, 0, True),       # groups of 32: one slot each
+    (100, 32, 2, 32, 2, 0, True),       # groups of one expert
+    (100, 64, 4, 32, 3, 0, True),       # groups of 2
+    (90, 40, 3, 5, 2, 0, True),         # groups of 8, the last slot partly empty
 ])
 def test_route_edges(moe, T, E, k, G, gpt, renorm, ties):
     rng = np.random.default_rng(T * 7 + E)
