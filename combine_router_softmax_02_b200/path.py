@@ -81,6 +81,14 @@ class DispatchCombine:
         return self.combine()
 
 
+def token_ranges(T: int, chunks: int):
+    """`chunks` contiguous, non-empty token ranges [a, b) covering [0, T) in
+    order, of sizes that differ by at most one (fewer when T < chunks)."""
+    n = max(1, min(chunks, T))
+    edges = [T * i // n for i in range(n + 1)]
+    return [(a, b) for a, b in zip(edges, edges[1:]) if b > a]
+
+
 class HostPipeline:
     """Steps of a DispatchCombine whose inputs and outputs are pinned host
     buffers, with the host<->device copies overlapped with the kernels.
@@ -107,9 +115,7 @@ class HostPipeline:
         self.logits = [torch.empty((T, E), dtype=torch.float32, device=dev) for _ in range(2)]
         self.x = [torch.empty((T, H), dtype=dc.dtype, device=dev) for _ in range(2)]
         self.out = [torch.empty((T, H), dtype=dc.out_dtype, device=dev) for _ in range(2)]
-        n = max(1, min(chunks, T))
-        edges = [T * i // n for i in range(n + 1)]
-        self.ranges = [(a, b) for a, b in zip(edges, edges[1:]) if b > a]
+        self.ranges = token_ranges(T, chunks)
         self.in_free = [None, None]   # kernels done with logits[b] and x[b]
         self.out_free = [None, None]  # copies out done with out[b]
         self.last = [None, None, None]  # last event of each stream
