@@ -1,7 +1,8 @@
 // Pieces of the layout shared by the layout kernel (build_layout.cu) and the
-// fused static-placement kernel (route_layout_static.cu): arguments, the
-// shared-memory plan, per-token pick loading, warp bin ballots, the grid
-// barrier, and the second phase that turns bin counts into rows.
+// one-launch front ends (route_layout_static.cu, route_assign_layout.cu):
+// arguments, the shared-memory plan, per-token pick loading, warp bin
+// ballots, the grid barrier (counted in rounds, so one launch can pass several),
+// and the two phases that turn picks into bin counts and bin counts into rows.
 //
 // One launch, two phases.  Every block owns a contiguous chunk of tokens.
 // Phase 1 counts the rows of every bin ("bins" are ranks for DEDUP, ranks then
