@@ -150,6 +150,43 @@ def step_bytes(cfg: W.Config, rows: int, rows_hop1: int, S: int) -> dict:
     return d
 
 
+def make_trace(cfg: W.Config, counts, expert_slot, expert_rank, rank_active, rank_offsets,
+               send_counts, group_offsets=None, calls=None) -> dict:
+    """One step's routing decisions and buffer sizes, from host arrays: the
+    replica chosen for every active expert, each rank's group, activated experts
+    and received rows, and the two all-to-all-v exchanges the layout stands for
+    (bytes per source -> destination rank), plus per-call start and duration
+    (us) when `calls` gives [(name, start_us, dur_us)]."""
+    b = cfg.H * cfg.elem_bytes
+    rpg = max(cfg.ranks_per_group, 1)
+    counts, expert_slot, expert_rank = (np.asarray(a) for a in (counts, expert_slot, expert_rank))
+    rows = np.diff(np.asarray(rank_offsets))
+    S = np.asarray(send_counts).reshape(cfg.R, cfg.R)
+    tr = {
+        "workload": cfg.name,
+        "ranks": cfg.R,
+        "replicas": [{"expert": int(e), "demand": int(counts[e]), "slot": int(expert_slot[e]),
+                      "rank": int(expert_rank[e])} for e in np.flatnonzero(counts > 0)],
+        "rank_detail": [{"rank": r, "group": r // rpg if cfg.mode == W.TWO_HOP else 0,
+                         "active_experts": int(rank_active[r]), "rows": int(rows[r]),
+                         "recv_bytes": int(rows[r]) * b} for r in range(cfg.R)],
+        "collectives": [
+            {"name": "dispatch all-to-all-v (pack: token rows to their destination ranks)",
+             "bytes": int(S.sum()) * b, "bytes_src_dst": (S * b).tolist()},
+            {"name": "combine all-to-all-v (expert outputs back to the token's rank)",
+             "bytes": int(S.sum()) * b, "bytes_src_dst": (S.T * b).tolist()},
+        ],
+    }
+    if cfg.mode == W.TWO_HOP and group_offsets is not None:
+        g_rows = np.diff(np.asarray(group_offsets))
+        tr["collectives"].insert(0, {"name": "dispatch hop 1 (token rows to their groups)",
+                                     "bytes": int(g_rows.sum()) * b,
+                                     "group_bytes": [int(x) * b for x in g_rows]})
+    if calls is not None:
+        tr["calls_us"] = [{"call": n, "start": round(t, 3), "duration": round(d, 3)} for n, t, d in calls]
+    return tr
+
+
 # ------------------------------------------------------------------- ours
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
@@ -308,6 +345,22 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     st = moe.get_status()
     if st != 0:
         raise RuntimeError(f"device status after statistics: {moe.status_string(st)}")
+    if args.trace:
+        last = evs[-1]
+        calls = [(n, last[0].elapsed_time(last[j]) * 1e3, last[j].elapsed_time(last[j + 1]) * 1e3)
+                 for j, n in enumerate(names)]
+        L = dc.layout
+        if args.fused and single:  # the single-replica kernel takes the ranks as given
+            e_slot = rm.replica_slots[rm.replica_offsets[:-1]]
+            e_rank = rm.slot_rank[e_slot]
+        else:
+            e_slot, e_rank = dc.expert_slot.cpu().numpy(), dc.expert_rank.cpu().numpy()
+        tr = make_trace(cfg, dc.counts.cpu().numpy(), e_slot, e_rank, dc.rank_active.cpu().numpy(),
+                        L.rank_offsets.cpu().numpy(), L.send_counts.cpu().numpy(),
+                        L.group_offsets.cpu().numpy() if cfg.mode == W.TWO_HOP else None, calls)
+        path = args.trace if world == 1 else f"{args.trace}.rank{rank}"
+        with open(path, "w") as f:
+            json.dump(tr, f)
 
     # whole-job aggregation: max time over ranks, rows summed over ranks
     agg = aggregate(dist, dev, [elapsed_ms, e2e_ms], [rows * args.steps, rows * e2e_steps])
@@ -482,6 +535,9 @@ def main(argv=None):
     ap.add_argument("--fused", action="store_true",
                     help="route, histogram, assignment and layout in one launch "
                          "(the single-replica kernel when every expert has one replica)")
+    ap.add_argument("--trace", default="",
+                    help="write the last timed step's routing decisions, buffer sizes and call "
+                         "times as JSON to this path (outside the timed region)")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of the step captured in a CUDA graph")
     args = ap.parse_args(argv)

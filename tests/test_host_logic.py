@@ -15,3 +15,32 @@ def test_token_ranges_cover_in_order(T, chunks):
     if r:
         sizes = [b - a for a, b in r]
         assert max(sizes) - min(sizes) <= 1
+
+
+def test_step_trace_structure():
+    """bench's step trace: replicas of active experts only, rows and bytes per
+    rank, and the dispatch/combine matrices, from a hand-made tiny layout."""
+    import numpy as np
+    import bench
+    import workloads as W
+    cfg = W.CONFIGS["c1"].with_(R=2, E=4, k=2, T=4)
+    counts = np.array([3, 0, 4, 1])
+    slot = np.array([0, -1, 5, 3])
+    rank = np.array([0, -1, 1, 1])
+    active = np.array([1, 2])
+    offsets = np.array([0, 3, 7])                # rank 0: 3 rows, rank 1: 4 rows
+    send = np.array([[2, 0], [1, 4]])            # rows by (source rank, destination rank)
+    tr = bench.make_trace(cfg, counts, slot, rank, active, offsets, send,
+                          calls=[("route_topk", 0.0, 5.0), ("pack", 5.0, 2.5)])
+    b = cfg.H * cfg.elem_bytes
+    assert [r["expert"] for r in tr["replicas"]] == [0, 2, 3]
+    assert tr["replicas"][1] == {"expert": 2, "demand": 4, "slot": 5, "rank": 1}
+    assert [d["rows"] for d in tr["rank_detail"]] == [3, 4]
+    assert tr["rank_detail"][1]["recv_bytes"] == 4 * b
+    disp, comb = tr["collectives"]
+    assert disp["bytes"] == comb["bytes"] == 7 * b
+    assert disp["bytes_src_dst"] == [[2 * b, 0], [1 * b, 4 * b]]
+    assert comb["bytes_src_dst"] == [[2 * b, 1 * b], [0, 4 * b]]  # combine reverses the direction
+    # the rows each rank receives equal the column sums of the send matrix
+    assert [sum(col) for col in zip(*disp["bytes_src_dst"])] == [d["recv_bytes"] for d in tr["rank_detail"]]
+    assert tr["calls_us"][1] == {"call": "pack", "start": 5.0, "duration": 2.5}
