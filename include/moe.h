@@ -177,9 +177,13 @@ MOE_API size_t moe_layout_workspace_size(int32_t T, int32_t k, int32_t E, int32_
  * topk_idx [T][k], topk_w [T][k], expert_rank [E] (from moe_replica_assign).
  * tokens_per_rank: source rank of token t is t / tokens_per_rank (< R).
  * workspace: device scratch of moe_layout_workspace_size() bytes, 16-byte
- * aligned; its contents on entry do not matter.  Fills every buffer of
- * `layout` and its shape fields.  Rows past layout->capacity are dropped (their
- * token_rows entries are -1) and set MOE_ERR_CAPACITY.
+ * aligned; its contents on entry do not matter.  It holds the launch's grid
+ * barrier, so calls whose executions overlap on the GPU (other streams, other
+ * host threads) need workspaces of their own.  The kernel is a cooperative
+ * launch sized to the blocks that fit on the GPU at once; its barrier waits
+ * are bounded (MOE_ERR_TIMEOUT).  Fills every buffer of `layout` and its shape
+ * fields.  Rows past layout->capacity are dropped (their token_rows entries
+ * are -1) and set MOE_ERR_CAPACITY.
  */
 MOE_API int moe_build_layout(const int32_t *topk_idx, const float *topk_w, const int32_t *expert_rank,
                      int32_t T, int32_t tokens_per_rank, int32_t k, int32_t E, int32_t R,
