@@ -46,8 +46,11 @@ cudaError_t launch_k(const LayoutArgs &a0, int kind, const DeviceCtx &ctx, cudaS
   if (err != cudaSuccess) return err;
   int resident = 0;
   if ((err = max_resident_blocks((const void *)kern, smem, ctx, resident)) != cudaSuccess) return err;
-  split_tokens(a.T, resident < kBlocksPerSm * ctx.num_sms ? resident : kBlocksPerSm * ctx.num_sms,
-               a.nblk, a.chunk);
+  // blocks per SM: a sweep over 1-4 picked 2 for DEDUP on the 65536-token
+  // workload (25.6 us against 28.8-29.0) and 1 for TWO_HOP on the two-hop one
+  // (28.9 us against 32.1-32.5)
+  const int bps = MODE == MOE_LAYOUT_TWO_HOP ? 1 : kBlocksPerSm;
+  split_tokens(a.T, resident < bps * ctx.num_sms ? resident : bps * ctx.num_sms, a.nblk, a.chunk);
   if ((err = cudaMemsetAsync(a.bar, 0, sizeof(int) * 16, s)) != cudaSuccess) return err;
   void *args[] = {&a, const_cast<DeviceCtx *>(&ctx)};
   err = cudaLaunchCooperativeKernel((const void *)kern, dim3(a.nblk), dim3(kTile), args, smem, s);
