@@ -44,3 +44,20 @@ def test_step_trace_structure():
     # the rows each rank receives equal the column sums of the send matrix
     assert [sum(col) for col in zip(*disp["bytes_src_dst"])] == [d["recv_bytes"] for d in tr["rank_detail"]]
     assert tr["calls_us"][1] == {"call": "pack", "start": 5.0, "duration": 2.5}
+
+
+def test_step_trace_two_hop_groups():
+    """The two-hop trace adds the hop-1 exchange (rows per group) before the
+    rank-level dispatch, and reports each rank's group."""
+    import numpy as np
+    import bench
+    import workloads as W
+    cfg = W.CONFIGS["c5"].with_(R=4, ranks_per_group=2, E=8, k=2, T=6)
+    b = cfg.H * cfg.elem_bytes
+    tr = bench.make_trace(cfg, np.ones(8, int), np.arange(8), np.arange(8) % 4, np.array([2, 2, 2, 2]),
+                          np.array([0, 2, 4, 7, 9]), np.ones((4, 4), int), group_offsets=np.array([0, 5, 8]))
+    hop1 = tr["collectives"][0]
+    assert hop1["name"].startswith("dispatch hop 1")
+    assert hop1["bytes"] == 8 * b and hop1["group_bytes"] == [5 * b, 3 * b]
+    assert [d["group"] for d in tr["rank_detail"]] == [0, 0, 1, 1]
+    assert "calls_us" not in tr
