@@ -182,7 +182,9 @@ def replica_assign(counts, replica_offsets, replica_slots, slot_rank, R: int):
 def optimal_max_active(counts, replica_offsets, replica_slots, slot_rank, R: int) -> int:
     """Brute force over every replica choice: the minimum possible max activated
     experts per rank (the "expensive optimal assignment" the page contrasts
-    with the greedy).  Tiny inputs only."""
+    with the greedy).  Tiny inputs only.  Pinned by hand-worked optima (one
+    where the greedy is strictly worse), the page's toy example and a
+    bipartite-matching optimum computed by a library routine."""
     active = [e for e in range(len(counts)) if counts[e] > 0]
     choices = [sorted({int(slot_rank[s]) for s in replica_slots[replica_offsets[e]:replica_offsets[e + 1]]})
                for e in active]

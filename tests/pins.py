@@ -215,6 +215,68 @@ def check_assign_brute(replica_assign, optimal_max_active, seed=6):
     return float(np.mean(gaps)) if gaps else 0.0
 
 
+def matching_optimum(counts, off, slots, slot_rank, R):
+    """The min-max number of activated experts per rank by a different route
+    than enumeration: the largest load m is feasible exactly when every active
+    expert can be matched to a distinct copy among m copies of each rank that
+    holds one of its replicas (a bipartite matching, scipy's library routine);
+    the answer is the smallest feasible m."""
+    from scipy.sparse import csr_matrix
+    from scipy.sparse.csgraph import maximum_bipartite_matching
+    active = [e for e in range(len(counts)) if counts[e] > 0]
+    if not active:
+        return 0
+    ranks = [sorted({int(slot_rank[s]) for s in slots[off[e]:off[e + 1]]}) for e in active]
+    for m in range(1, len(active) + 1):
+        rows, cols = [], []
+        for i, rs in enumerate(ranks):
+            for r in rs:
+                for c in range(m):
+                    rows.append(i)
+                    cols.append(r * m + c)
+        g = csr_matrix((np.ones(len(rows)), (rows, cols)), shape=(len(active), R * m))
+        match = maximum_bipartite_matching(g, perm_type="column")
+        if np.all(match >= 0):
+            return m
+    raise AssertionError("no feasible load: an active expert without a replica")
+
+
+def check_optimal_max_active(optimal_max_active, replica_assign, seed=11):
+    """The brute-force optimum against the hand-worked fixtures (one where the
+    greedy is strictly worse, one above the counting bound), the page's toy
+    (optimum 1), and a bipartite-matching optimum on random tiny maps; and
+    always ceil(A/R) <= optimum <= greedy."""
+    for inst in golden("metro_optimum_hand.json")["instances"]:
+        args = (np.asarray(inst["counts"]), np.asarray(inst["replica_offsets"]),
+                np.asarray(inst["replica_slots"]), np.asarray(inst["slot_rank"]), inst["R"])
+        assert optimal_max_active(*args) == inst["optimum"], inst["name"]
+        _, _, act = replica_assign(*args)
+        assert act.tolist() == inst["greedy_rank_active"], inst["name"]
+        assert int(act.max()) == inst["greedy_max_active"]
+    g, counts, off, slots, sr, R = toy_instance()
+    assert optimal_max_active(counts, off, slots, sr, R) == g["metro_max_active_per_gpu"] == 1
+    rng = np.random.default_rng(seed)
+    strictly_worse = 0
+    for _ in range(150):
+        E, R = int(rng.integers(1, 8)), int(rng.integers(1, 5))
+        reps = [rng.choice(R, size=int(rng.integers(1, min(R, 3) + 1)), replace=False).tolist()
+                for _ in range(E)]
+        off = np.zeros(E + 1, np.int64)
+        off[1:] = np.cumsum([len(r) for r in reps])
+        sr = np.asarray([r for rr in reps for r in rr], np.int64)
+        slots = rng.permutation(sr.shape[0])          # slot ids unrelated to their position
+        sr = sr[np.argsort(slots)]                      # slot_rank indexed by slot id
+        counts = rng.integers(0, 3, size=E)
+        opt = optimal_max_active(counts, off, slots, sr, R)
+        assert opt == matching_optimum(counts, off, slots, sr, R)
+        A = int(np.count_nonzero(counts))
+        assert -(-A // R) <= opt
+        _, _, act = replica_assign(counts, off, slots, sr, R)
+        assert opt <= int(act.max(initial=0))
+        strictly_worse += int(act.max(initial=0)) > opt
+    return strictly_worse
+
+
 # --------------------------------------------------------------- layout ----
 def brute_layout(idx, w, expert_rank, tokens_per_rank, R, mode, rpg=0):
     """Pure-Python layout straight from the row definitions."""

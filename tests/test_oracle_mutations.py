@@ -176,3 +176,46 @@ def test_placement_ignoring_affinity_caught():
         return oracle.correlated_placement(np.zeros_like(C), counts, R)
     with pytest.raises(AssertionError):
         pins.check_placement(mutant)
+
+
+def _opt_zero(counts, off, slots, sr, R):
+    return 0
+
+
+def _opt_max_over_choices(counts, off, slots, sr, R):
+    # the worst choice instead of the best
+    import itertools
+    active = [e for e in range(len(counts)) if counts[e] > 0]
+    ch = [sorted({int(sr[s]) for s in slots[off[e]:off[e + 1]]}) for e in active]
+    return max((int(np.bincount(np.asarray(p, np.int64), minlength=R).max()) for p in itertools.product(*ch)),
+               default=0)
+
+
+def _opt_first_replica(counts, off, slots, sr, R):
+    # no choice at all: every active expert on its first listed replica
+    load = np.zeros(R, np.int64)
+    for e in range(len(counts)):
+        if counts[e] > 0:
+            load[sr[slots[off[e]]]] += 1
+    return int(load.max())
+
+
+def _opt_counting_bound(counts, off, slots, sr, R):
+    return -(-int(np.count_nonzero(counts)) // R)
+
+
+def _opt_counts_inactive(counts, off, slots, sr, R):
+    # inactive experts treated as active
+    return oracle.optimal_max_active(np.ones(len(counts), np.int64), off, slots, sr, R)
+
+
+def _opt_slot_as_rank(counts, off, slots, sr, R):
+    # the slot id taken for the rank
+    return oracle.optimal_max_active(counts, off, slots, np.arange(int(np.max(slots)) + 1) % max(R, 1), R)
+
+
+@pytest.mark.parametrize("mutant", [_opt_zero, _opt_max_over_choices, _opt_first_replica,
+                                    _opt_counting_bound, _opt_counts_inactive, _opt_slot_as_rank])
+def test_optimal_max_active_mutants_caught(mutant):
+    with pytest.raises(AssertionError):
+        pins.check_optimal_max_active(mutant, oracle.replica_assign)

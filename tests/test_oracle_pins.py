@@ -124,3 +124,9 @@ def test_derived_placement_shrinks_dedup_rows():
         rows[name] = int(oracle.build_layout(idx, w, rank, cfg.tokens_per_rank, cfg.R, oracle.DEDUP)["num_rows"])
     assert rows["derived"] < rows["roundrobin"]
     assert rows["derived"] <= 1.02 * rows["block"]      # close to the planted clusters
+
+
+def test_optimal_max_active_pinned():
+    # the greedy is strictly worse than the optimum on some random tiny maps,
+    # as the page's "within 10.9%" implies it can be
+    assert pins.check_optimal_max_active(oracle.optimal_max_active, oracle.replica_assign) > 0
