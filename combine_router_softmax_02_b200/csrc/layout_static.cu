@@ -17,13 +17,18 @@ std::mutex g_scratch_mu;
 
 // Device address of g_layout_scratch on the current device.  In host code the
 // array's name is only a stand-in, so the address comes from the runtime,
-// once per device, with that device current.
-int scratch_address(void **out) {
+// once per device, with that device current.  The lookup is not a stream
+// operation and may load the module, so it is refused while `stream` is being
+// captured: the first call on a device must come before any capture.
+int scratch_address(cudaStream_t stream, void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_ptr[dev]) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return MOE_ERR_UNSUPPORTED;
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
     g_scratch_ptr[dev] = p;
@@ -43,7 +48,7 @@ extern "C" int moe_build_layout_static(const int32_t *topk_idx, const float *top
   if (need == 0 && T > 0) return MOE_ERR_INVALID_ARG;
   if (need > MOE_LAYOUT_STATIC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
   void *scratch = nullptr;
-  const int rc = scratch_address(&scratch);
+  const int rc = scratch_address(reinterpret_cast<cudaStream_t>(stream), &scratch);
   if (rc != MOE_OK) return rc;
   // Same checks and kernels as moe_build_layout; the launch clears the parts
   // of the scratch that must start at zero.

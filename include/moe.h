@@ -24,6 +24,10 @@
  *   (bad index in an input, capacity exceeded, a bounded wait that ran out)
  *   are recorded in a per-device status word (first error wins), and the
  *   offending element is skipped; moe_get_status() reads and clears it.
+ * - The library keeps, per device, the device addresses of its own status
+ *   word (and of the scratch array of moe_build_layout_static), looked up on
+ *   the first call on that device.  It is not usable across cudaDeviceReset:
+ *   a reset destroys the context those addresses belong to.
  * - Limits: 1 <= E <= 1024; 1 <= k <= min(E, 16); 1 <= R <= 64;
  *   T * k < 2^31; replica slots S <= 32768; H * element size a multiple of
  *   16 bytes; n_groups <= 32.
@@ -207,9 +211,11 @@ MOE_API int moe_build_layout(const int32_t *topk_idx, const float *topk_w, const
  * Returns MOE_ERR_UNSUPPORTED, before anything is launched, when
  * moe_layout_workspace_size() for these sizes exceeds
  * MOE_LAYOUT_STATIC_SCRATCH_BYTES (for example 65536 tokens over 64 ranks
- * needs 135 KB in DEDUP mode).  The first call on a device looks up the
- * array's device address with that device current; make that first call
- * before any stream capture.  All calls share the one array, whose contents
+ * needs 135 KB in DEDUP mode; 65536 tokens over 256 experts, 528 KB in
+ * PER_PICK mode).  The first call on a device looks up the array's device
+ * address with that device current and keeps it; make that first call before
+ * any stream capture (a first call on a capturing stream returns
+ * MOE_ERR_UNSUPPORTED and launches nothing).  All calls share the one array, whose contents
  * persist from call to call (each call clears what must start at zero):
  * calls whose executions overlap on the GPU -- on different streams, or from
  * different host threads -- race on it and must be serialised by the caller.

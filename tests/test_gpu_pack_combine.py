@@ -38,6 +38,53 @@ def check_combine_sampled(out_dev, y_rows_f64, token_rows, coef, tokens, fmt):
     assert_close_combine(got, ref, absum, fmt)
 
 
+class PackedRows:
+    """The oracle's packed rows ``Y[i] = X[row_token[i]]`` (identity experts)
+    as float64, gathered on demand so that a full-size combine can run in
+    token chunks without holding every row at once."""
+
+    def __init__(self, x64_of, row_token, H):
+        self.x64_of, self.row_token, self.shape = x64_of, np.asarray(row_token, np.int64), (len(row_token), H)
+
+    def __getitem__(self, rows):
+        return self.x64_of(self.row_token[rows])
+
+
+def assert_rows_bit_exact(dev_rows, x_bits, row_token, chunk=32768):
+    """Every packed row on the device equals the oracle's pack of the token
+    bits, compared in chunks of rows copied back to the host."""
+    n = len(row_token)
+    for r0 in range(0, n, chunk):
+        r1 = min(n, r0 + chunk)
+        got = bits(dev_rows[r0:r1])
+        want = oracle.pack(x_bits, row_token[r0:r1])
+        if not np.array_equal(got, want):
+            bad = np.flatnonzero(np.any(got != want, axis=1))
+            raise AssertionError(f"{len(bad)} packed rows differ in rows [{r0}, {r1}); first {r0 + bad[0]}")
+
+
+def check_combine_all_tokens(out_dev, y, token_rows, coef, fmt, chunk=4096):
+    """Oracle combine of every token, in token chunks, against the device output."""
+    T = token_rows.shape[0]
+    c = np.asarray(coef, np.float64)
+    for t0 in range(0, T, chunk):
+        toks = np.arange(t0, min(T, t0 + chunk))
+        ref = oracle.combine(y, token_rows, c, tokens=toks)
+        absum = oracle.combine(_Abs(y), token_rows, np.abs(c), tokens=toks)
+        got = out_dev[t0:t0 + len(toks)].double().cpu().numpy()
+        assert_close_combine(got, ref, absum, fmt, what=f"combine tokens [{t0}, {t0 + len(toks)})")
+
+
+class _Abs:
+    """|Y| of a row source, for the bound's sum of absolute terms."""
+
+    def __init__(self, y):
+        self.y, self.shape = y, y.shape
+
+    def __getitem__(self, rows):
+        return np.abs(np.asarray(self.y[rows], np.float64))
+
+
 SMALL = [("c1", W.DEDUP), ("c1", W.PER_PICK), ("c2", W.DEDUP), ("c3", W.DEDUP), ("c3", W.PER_PICK)]
 
 
@@ -120,32 +167,16 @@ def test_conservation_and_all_ones(moe):
         assert moe.get_status() == 0
 
 
-def check_two_hop(moe, cfg, sample=None):
-    case = Case(cfg)
-    ref = case.oracle_route()
-    RL = ref["layout"]
-    dc = case.device_path(moe)
-    x = case.x_cpu.cuda()
-    out = dc.step(to_dev(case.logits), x)
-    assert moe.get_status() == 0
-    lay = layout_fields(dc.layout, W.TWO_HOP)
-    assert_layout_equal(lay, RL, W.TWO_HOP, w_tol=row_coef_tol(case.logits, ref["idx"], cfg.k))
-    n, n1 = lay["num_rows"], lay["num_rows_hop1"]
-    xb = bits(case.x_cpu)
-    r1 = np.arange(n1) if sample is None else W.sample_indices(n1, sample, 1)
-    r2 = np.arange(n) if sample is None else W.sample_indices(n, sample, 2)
-    assert np.array_equal(bits(dc.packed_hop1[torch.from_numpy(r1).cuda()]), xb[RL["hop1_row_token"][r1]])
-    assert np.array_equal(bits(dc.packed[torch.from_numpy(r2).cuda()]), xb[RL["row_token"][r2]])
-    # combine in reverse: group partials rounded to the wire dtype, then summed
-    toks = np.arange(cfg.T) if sample is None else W.sample_indices(cfg.T, sample, 3)
-    x64 = case.x_cpu.double().numpy()
-    fmt = fmt_of(dc.out_dtype)
+def check_two_hop_tokens(out, hop1_buf, RL, x_of, toks, fmt):
+    """Two-hop combine of the tokens `toks` against the oracle: each group's
+    rank rows summed and rounded to the wire dtype, then the groups summed;
+    and the stored group partials of those tokens, each within its own bound."""
     tr, tg = RL["token_rows"][toks], RL["token_groups"][toks]
     used2, used1 = np.unique(tr[tr >= 0]), np.unique(tg[tg >= 0])
     sub = {"token_rows": np.where(tr >= 0, np.searchsorted(used2, tr), -1),
            "token_groups": np.where(tg >= 0, np.searchsorted(used1, tg), -1),
            "hop2_src_row": np.searchsorted(used1, RL["hop2_src_row"][used2])}
-    y2 = x64[RL["row_token"][used2]]
+    y2 = x_of(RL["row_token"][used2])
     c2 = RL["row_coef"][used2]
     o, zs = oracle.combine_two_hop(y2, sub, c2, fmt)
     absum, _ = oracle.combine_two_hop(np.abs(y2), sub, np.abs(c2), "f32")
@@ -158,13 +189,36 @@ def check_two_hop(moe, cfg, sample=None):
             extra[have] += oracle.ulp(z, fmt)
     assert_close_combine(out[torch.from_numpy(toks).cuda()].double().cpu().numpy(), o, absum, fmt,
                          extra=extra, what="two-hop combine")
-    # the stored group partials: each within its own bound of the oracle's rounded partial
-    z_dev = dc.hop1_buf[torch.from_numpy(used1.astype(np.int64)).cuda()].double().cpu().numpy()
+    z_dev = hop1_buf[torch.from_numpy(used1.astype(np.int64)).cuda()].double().cpu().numpy()
     z_ref = np.stack([zs[i] for i in range(len(used1))])
     zabs = np.zeros_like(z_ref)
     for i2, s1 in enumerate(sub["hop2_src_row"]):
         zabs[s1] += np.abs(c2[i2] * y2[i2])
     assert_close_combine(z_dev, z_ref, zabs, fmt, extra=oracle.ulp(z_ref, fmt), what="group partials")
+
+
+def check_two_hop(moe, cfg, chunk=4096):
+    """The two-hop path against the oracle: layout bit-exact, every hop-1 and
+    hop-2 packed row bit-exact, every token's combine and group partial
+    within its bound (in token chunks)."""
+    case = Case(cfg)
+    ref = case.oracle_route()
+    RL = ref["layout"]
+    dc = case.device_path(moe)
+    x = case.x_cpu.cuda()
+    out = dc.step(to_dev(case.logits), x)
+    assert moe.get_status() == 0
+    lay = layout_fields(dc.layout, W.TWO_HOP)
+    assert_layout_equal(lay, RL, W.TWO_HOP, w_tol=row_coef_tol(case.logits, ref["idx"], cfg.k))
+    n, n1 = lay["num_rows"], lay["num_rows_hop1"]
+    xb = bits(case.x_cpu)
+    assert_rows_bit_exact(dc.packed_hop1[:n1], xb, RL["hop1_row_token"])
+    assert_rows_bit_exact(dc.packed[:n], xb, RL["row_token"])
+    fmt = fmt_of(dc.out_dtype)
+    xs = case.x_cpu
+    x_of = lambda t: xs[torch.from_numpy(np.asarray(t, np.int64))].double().numpy()  # noqa: E731
+    for t0 in range(0, cfg.T, chunk):
+        check_two_hop_tokens(out, dc.hop1_buf, RL, x_of, np.arange(t0, min(cfg.T, t0 + chunk)), fmt)
     # not storing the partials changes nothing else
     out2 = moe.combine(dc.packed, dc.layout, out_dtype=dc.out_dtype, store_hop1=False)
     assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
@@ -175,14 +229,15 @@ def test_two_hop_small_every_row(moe):
     check_two_hop(moe, W.CONFIGS["c5"].with_(T=2048))
 
 
-def test_two_hop_full_size_sampled(moe):
-    check_two_hop(moe, W.CONFIGS["c5"], sample=3000)
+def test_two_hop_full_size_every_row(moe):
+    """The two-hop benchmark workload (32768 tokens x 4096 bf16) in full."""
+    check_two_hop(moe, W.CONFIGS["c5"])
 
 
-def test_full_size_prefill_path_sampled(moe):
+def test_full_size_prefill_path_every_row(moe):
     """The benchmark's workload and launch configuration (DispatchCombine.step
-    on 65536 tokens x 7168 bf16): layout bit-exact, sampled packed rows
-    bit-exact, sampled output tokens within the combine bound."""
+    on 65536 tokens x 7168 bf16): layout bit-exact, every packed row bit-exact,
+    every output token within the combine bound."""
     cfg = W.CONFIGS["c4"]
     case = Case(cfg)
     ref = case.oracle_route()
@@ -194,11 +249,7 @@ def test_full_size_prefill_path_sampled(moe):
     assert np.array_equal(dc.topk_idx.cpu().numpy(), ref["idx"])
     lay = layout_fields(dc.layout, W.DEDUP)
     assert_layout_equal(lay, RL, W.DEDUP, w_tol=row_coef_tol(case.logits, ref["idx"], cfg.k))
-    rows = W.sample_indices(lay["num_rows"], 4000, 5)
-    assert np.array_equal(bits(dc.packed[torch.from_numpy(rows).cuda()]),
-                          bits(case.x_cpu[torch.from_numpy(RL["row_token"][rows].astype(np.int64))]))
-    toks = W.sample_indices(cfg.T, 2000, 6)
+    assert_rows_bit_exact(dc.packed[:lay["num_rows"]], bits(case.x_cpu), RL["row_token"])
     xs = case.x_cpu
-    rt = RL["row_token"]
-    check_combine_sampled(out, lambda r: xs[torch.from_numpy(rt[r].astype(np.int64))].double().numpy(),
-                          RL["token_rows"], RL["row_coef"], toks, "bf16")
+    y = PackedRows(lambda t: xs[torch.from_numpy(t)].double().numpy(), RL["row_token"], cfg.H)
+    check_combine_all_tokens(out, y, RL["token_rows"], RL["row_coef"], "bf16")
