@@ -598,9 +598,12 @@ __device__ __forceinline__ void publish_counts(const LayoutArgs &a, const SmemPl
     for (int i = threadIdx.x; i < a.R * a.R; i += kTile) a.L.send_counts[i] = 0;
 }
 
-// Clears the block's shared counters and loads the expert -> rank map.
-__device__ __forceinline__ void smem_init(const LayoutArgs &a, const SmemPlan &P, int *sm) {
-  for (int i = threadIdx.x; i < a.E; i += kTile) sm[P.er + i] = __ldcg(a.expert_rank + i);
+// Clears the block's shared counters and loads the expert -> rank map (unless
+// the caller has already put it in shared memory: `load_er` false).
+__device__ __forceinline__ void smem_init(const LayoutArgs &a, const SmemPlan &P, int *sm,
+                                          bool load_er = true) {
+  if (load_er)
+    for (int i = threadIdx.x; i < a.E; i += kTile) sm[P.er + i] = __ldcg(a.expert_rank + i);
   for (int i = threadIdx.x; i < a.NBp; i += kTile) sm[P.cnt + i] = 0;
   for (int i = threadIdx.x; i < a.R * a.R; i += kTile) sm[P.send + i] = 0;
   __syncthreads();

@@ -1,4 +1,5 @@
-// METRO greedy replica assignment, one CTA: the kernel around metro_assign
+// METRO greedy replica assignment, one CTA: the kernel around metro_stage and
+// metro_solve
 // (assign_common.cuh, which states the algorithm and its sources).
 #include "assign_common.cuh"
 
@@ -11,9 +12,9 @@ __global__ void __launch_bounds__(256) replica_assign_kernel(
     int *__restrict__ expert_slot, int *__restrict__ expert_rank, int *__restrict__ rank_active,
     DeviceCtx ctx) {
   extern __shared__ int sm[];
-  __shared__ int s_active[kMaxR];
-  metro_assign(counts, E, off, slots, n_entries, slot_rank, S, R, expert_slot, expert_rank,
-               rank_active, sm, s_active, ctx);
+  const MetroPlan P = metro_plan(E, n_entries, R);
+  metro_stage(E, off, slots, n_entries, slot_rank, S, R, sm, P);
+  metro_solve(counts, E, R, sm, P, sm + P.total, true, expert_slot, expert_rank, rank_active, ctx);
 }
 
 }  // namespace
@@ -22,10 +23,11 @@ cudaError_t launch_replica_assign(const int *counts, int E, const int *off, cons
                                   int n_entries, const int *slot_rank, int S, int R,
                                   int *expert_slot, int *expert_rank, int *rank_active,
                                   const DeviceCtx &ctx, cudaStream_t s) {
-  const size_t smem = sizeof(int) * ((size_t)2 * E + 1 + n_entries);
+  // the plan, then the expert -> rank map the walk leaves in shared memory
+  const size_t smem = sizeof(int) * ((size_t)assign_smem_ints(E, n_entries, R) + E);
   static std::atomic<unsigned long long> done{0};
-  cudaError_t err = set_smem_limit_once(replica_assign_kernel,
-                                        (int)(sizeof(int) * (2 * kMaxE + 1 + kMaxSlots)), done);
+  cudaError_t err = set_smem_limit_once(
+      replica_assign_kernel, (int)(sizeof(int) * (assign_smem_ints(kMaxE, kMaxSlots, kMaxR) + kMaxE)), done);
   if (err != cudaSuccess) return err;
   replica_assign_kernel<<<1, 256, smem, s>>>(counts, E, off, slots, n_entries, slot_rank, S, R,
                                              expert_slot, expert_rank, rank_active, ctx);

@@ -3,13 +3,16 @@
 // "METRO AllGather vs AllToAll for MoE decode" (fanout.sh): at decode sizes the
 // per-kernel launch cost is the price of the global routing information
 // (section "changes the routing information"), so the whole front end runs
-// as one cooperative kernel with four phases separated by grid barriers:
-//   A. every block routes the tokens of its chunk (route_common.cuh) and adds
-//      its demand histogram into the workspace's demand scratch;
-//   B. block 0 runs the METRO greedy (assign_common.cuh) over the complete
-//      demand vector: expert_slot, expert_rank, rank_active, counts;
-//   C. every block counts its chunk's layout bins with the assigned ranks;
-//   D. every block writes its rows (layout_common.cuh).
+// as one cooperative kernel in three phases separated by grid barriers:
+//   A. every block routes the tokens of its chunk (route_common.cuh), adds its
+//      demand histogram into the workspace's demand scratch, and stages the
+//      replica map in shared memory (assign_common.cuh, metro_stage);
+//   B. every block runs the METRO greedy over the complete demand vector into
+//      its own shared memory (the greedy is deterministic, so every block gets
+//      the same expert -> rank map and no block waits for another); block 0
+//      writes expert_slot, expert_rank, rank_active and counts; then every
+//      block counts its chunk's layout bins with that map;
+//   C. after the layout's barrier every block writes its rows (layout_common.cuh).
 // Every output equals that of moe_route_topk, moe_demand_hist,
 // moe_replica_assign and moe_build_layout called one after the other.
 #include "assign_common.cuh"
@@ -37,15 +40,24 @@ struct FrontArgs {
   int *rank_active;  // [R]
 };
 
+// METRO's shared memory starts after the expert -> rank map (the layout
+// plan's first region), which the greedy fills and the layout phases read.
+__host__ __device__ inline int front_smem_ints(int E, int NBp, int R, int n_entries) {
+  const int E4 = (E + 3) & ~3;
+  const int lay = layout::smem_plan(E, NBp, R, true).total, metro = E4 + metro_plan(E, n_entries, R).total;
+  return lay > metro ? lay : metro;
+}
+
 template <int EPL, bool FULL, int KM>
 __global__ void __launch_bounds__(kTile) route_assign_layout_kernel(FrontArgs f, LayoutArgs a, DeviceCtx ctx) {
   extern __shared__ int4 smem_raw[];
   int *sm = reinterpret_cast<int *>(smem_raw);
-  __shared__ __align__(16) uint32_t s_ck[kWarps][32];
+  __shared__ __align__(16) float s_cv[kWarps][32];
   __shared__ int s_ce[kWarps][32];
-  __shared__ int s_active[kMaxR];
   __shared__ int s_flag;
   const SmemPlan P = layout::smem_plan(a.E, a.NBp, a.R, true);
+  const MetroPlan M = metro_plan(a.E, f.n_entries, a.R);
+  int *smm = sm + ((a.E + 3) & ~3);  // METRO's scratch (P.er is the first region)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int *s_hist = sm + P.hist;
   for (int i = tid; i < a.E; i += kTile) s_hist[i] = 0;
@@ -60,7 +72,7 @@ __global__ void __launch_bounds__(kTile) route_assign_layout_kernel(FrontArgs f,
     int e;
     float w;
     route::route_token<EPL, FULL>(f.logits + (size_t)t * a.E, a.E, a.k, f.n_groups, f.gpt, f.renorm, L,
-                                  s_ck[warp], s_ce[warp], lane, e, w, bad);
+                                  s_cv[warp], s_ce[warp], lane, e, w, bad);
     if (lane < a.k) {
       f.idx_out[(size_t)t * a.k + lane] = e;
       f.w_out[(size_t)t * a.k + lane] = w;
@@ -71,25 +83,24 @@ __global__ void __launch_bounds__(kTile) route_assign_layout_kernel(FrontArgs f,
   __syncthreads();
   for (int i = tid; i < a.E; i += kTile)
     if (s_hist[i]) atomicAdd(&a.cnt[i], s_hist[i]);
+  __syncthreads();  // s_hist is read out before the replica map reuses its memory
+  metro_stage(a.E, f.off, f.slots, f.n_entries, f.slot_rank, f.S, a.R, smm, M);
   if (!layout::grid_barrier(a, ctx, &s_flag, 1)) return;
 
-  // B: one block assigns every active expert to a replica (its shared memory
-  // is free until phase C)
-  if (blockIdx.x == 0) {
-    metro_assign(a.cnt, a.E, f.off, f.slots, f.n_entries, f.slot_rank, f.S, a.R, f.expert_slot,
-                 f.expert_rank, f.rank_active, sm, s_active, ctx);
+  // B: the greedy in every block, straight into the layout's expert -> rank map
+  metro_solve(a.cnt, a.E, a.R, smm, M, sm + P.er, blockIdx.x == 0, f.expert_slot, f.expert_rank,
+              f.rank_active, ctx);
+  if (blockIdx.x == 0)
     for (int i = tid; i < a.E; i += kTile) f.counts[i] = __ldcg(a.cnt + i);
-  }
-  if (!layout::grid_barrier(a, ctx, &s_flag, 2)) return;
 
-  // C + D: the layout with the assigned ranks
-  layout::smem_init(a, P, sm);
+  // B + C: the layout with the assigned ranks
+  layout::smem_init(a, P, sm, false);
   if (a.mode == MOE_LAYOUT_DEDUP)
-    layout::layout_phases<KM, MOE_LAYOUT_DEDUP>(a, P, sm, t0, t1, ctx, &s_flag, 3);
+    layout::layout_phases<KM, MOE_LAYOUT_DEDUP>(a, P, sm, t0, t1, ctx, &s_flag, 2);
   else if (a.mode == MOE_LAYOUT_TWO_HOP)
-    layout::layout_phases<KM, MOE_LAYOUT_TWO_HOP>(a, P, sm, t0, t1, ctx, &s_flag, 3);
+    layout::layout_phases<KM, MOE_LAYOUT_TWO_HOP>(a, P, sm, t0, t1, ctx, &s_flag, 2);
   else
-    layout::layout_phases<KM, MOE_LAYOUT_PER_PICK>(a, P, sm, t0, t1, ctx, &s_flag, 3);
+    layout::layout_phases<KM, MOE_LAYOUT_PER_PICK>(a, P, sm, t0, t1, ctx, &s_flag, 2);
 }
 
 std::atomic<unsigned long long> g_smem_set[6][2][2];
@@ -99,8 +110,7 @@ cudaError_t launch_front(const FrontArgs &f0, const LayoutArgs &a0, int slot, co
                          cudaStream_t s) {
   FrontArgs f = f0;
   LayoutArgs a = a0;
-  const int ints = max(layout::smem_plan(a.E, a.NBp, a.R, true).total, assign_smem_ints(a.E, f.n_entries));
-  const size_t smem = sizeof(int) * (size_t)ints;
+  const size_t smem = sizeof(int) * (size_t)front_smem_ints(a.E, a.NBp, a.R, f.n_entries);
   auto kern = route_assign_layout_kernel<EPL, FULL, KM>;
   cudaError_t err = set_smem_limit_once(kern, kFrontSmemMax, g_smem_set[slot][FULL][KM > 8]);
   if (err != cudaSuccess) return err;
@@ -129,8 +139,7 @@ cudaError_t launch_epl(const FrontArgs &f, const LayoutArgs &a, int slot, const 
 size_t front_smem_bytes(int E, int k, int R, int rpg, int mode, int n_entries) {
   (void)k;
   const int NBp = (layout::num_bins(E, R, mode == MOE_LAYOUT_TWO_HOP ? rpg : 1, mode) + 3) & ~3;
-  const int ints = max(layout::smem_plan(E, NBp, R, true).total, assign_smem_ints(E, n_entries));
-  return sizeof(int) * (size_t)ints;
+  return sizeof(int) * (size_t)front_smem_ints(E, NBp, R, n_entries);
 }
 
 cudaError_t launch_route_assign_layout(const float *logits, int T, int E, int k, int n_groups, int gpt,

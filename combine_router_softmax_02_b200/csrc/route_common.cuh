@@ -7,9 +7,9 @@
 // editorial (lyndhub), section "The core problem".
 //
 // Lane l holds experts l, l+32, l+64, ... of its token (coalesced 128-byte
-// loads).  Selection works on an order-preserving u32 key of each logit; the
-// softmax maximum is the largest key, and the softmax sum a butterfly
-// reduction, so every lane ends with bit-identical values.
+// loads).  Each lane's largest logit becomes an order-preserving u32 key, so
+// the softmax maximum is one integer warp reduction; the softmax sum is a
+// butterfly reduction, so every lane ends with bit-identical values.
 //
 // Selection: the k-th largest of the 32 lane maxima (tau) is a lower bound on
 // the k-th largest key, so only the few elements at or above it can be picked.
@@ -76,31 +76,30 @@ struct Lanes {
 };
 
 // Routes the token whose logits start at `row`.  Lanes r < k return pick r in
-// (my_e, my_w); `bad` is set on lanes that saw a non-finite logit.  s_ck and
-// s_ce are this warp's 32-entry shared-memory candidate buffers (s_ck
+// (my_e, my_w); `bad` is set on lanes that saw a non-finite logit.  s_cv and
+// s_ce are this warp's 32-entry shared-memory candidate buffers (s_cv
 // 16-byte aligned).
 template <int EPL, bool FULL>
 __device__ __forceinline__ void route_token(const float *row, int E, int k, int n_groups, int gpt,
-                                            int renorm, const Lanes<EPL, FULL> &L, uint32_t *s_ck,
+                                            int renorm, const Lanes<EPL, FULL> &L, float *s_cv,
                                             int *s_ce, int lane, int &my_e, float &my_w,
                                             bool &bad) {
+  constexpr float kNoCand = -INFINITY;  // an empty slot, or an expert ruled out by its group
   float v[EPL];
-  uint32_t key[EPL];
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) v[j] = L.ok(j) ? __ldcs(row + lane + 32 * j) : 0.0f;
-  uint32_t kmax = 0, kmin = 0xffffffffu;
+  for (int j = 0; j < EPL; ++j) v[j] = L.ok(j) ? __ldcs(row + lane + 32 * j) : kNoCand;
+  // x * 0 is +-0 for finite x and NaN for an infinity or a NaN
+  float z = 0.0f, lmf = kNoCand;
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
-    key[j] = L.ok(j) ? order_key(v[j]) : 0u;
-    if (L.ok(j)) {
-      kmax = max(kmax, key[j]);
-      kmin = min(kmin, key[j]);
-    }
+    if (L.ok(j)) z = fmaf(v[j], 0.0f, z);
+    lmf = fmaxf(lmf, v[j]);
   }
-  bad |= kmax >= 0xff800000u || kmin < 0x00800000u;
+  bad |= !(z == 0.0f);
 
-  // softmax maximum and sum over all experts
-  const uint32_t top = __reduce_max_sync(kFull, kmax);
+  // softmax maximum and sum over all experts; only the lane maxima need keys
+  uint32_t lm = lmf == kNoCand ? 0u : order_key(lmf);  // this lane's largest selectable key
+  const uint32_t top = __reduce_max_sync(kFull, lm);
   const float m = key_value(top);
   float s = 0.0f;
 #pragma unroll
@@ -108,17 +107,16 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
     if (L.ok(j)) s += expf(v[j] - m);
   s = warp_sum(s);
 
-  uint32_t lm = kmax;  // this lane's largest selectable key
-  bool fresh = true;   // lm still equals kmax (then the warp max is `top`)
+  bool fresh = true;  // lm is still the lane maximum (then the warp max is `top`)
   if (L.limit) {
     // group score = largest logit in the group; lane g holds group g's key
     uint32_t gkey = 0;
     for (int g = 0; g < n_groups; ++g) {
-      uint32_t best = 0;
+      float bf = kNoCand;
 #pragma unroll
       for (int j = 0; j < EPL; ++j)
-        if (L.ok(j) && L.group(lane + 32 * j) == g) best = max(best, key[j]);
-      best = __reduce_max_sync(kFull, best);
+        if (L.ok(j) && L.group(lane + 32 * j) == g) bf = fmaxf(bf, v[j]);
+      const uint32_t best = __reduce_max_sync(kFull, bf == kNoCand ? 0u : order_key(bf));
       if (lane == g) gkey = best;
     }
     uint32_t keep = 0;
@@ -129,92 +127,98 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
       keep |= 1u << g;
       if (lane == g) gkey = 0;
     }
-    lm = 0;
+    lmf = kNoCand;
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
-      if (!(keep >> L.group(lane + 32 * j) & 1u)) key[j] = 0;  // 0 = not a candidate
-      lm = max(lm, key[j]);
+      if (!(keep >> L.group(lane + 32 * j) & 1u)) v[j] = kNoCand;
+      lmf = fmaxf(lmf, v[j]);
     }
+    lm = lmf == kNoCand ? 0u : order_key(lmf);
     fresh = false;
   }
 
   // Candidates.  tau = the k-th largest of the 32 lane maxima: k distinct
-  // elements reach it, so every top-k element has key >= tau.
+  // elements reach it, so every top-k element has a logit >= tau (tau == 0:
+  // fewer than k lanes hold a selectable expert; every slot is a candidate).
   uint32_t tau = 0;
   for (int r = 0; r < k; ++r) {
     tau = (r == 0 && fresh) ? top : __reduce_max_sync(kFull, lm);
     const unsigned b = __ballot_sync(kFull, lm == tau);
     if (lane == 31 - __clz(b)) lm = 0;  // any one lane holding the value
   }
+  const float tau_v = key_value(tau);
 
   // compaction in ascending expert order: slot j of lane l is expert l + 32 j
   const unsigned below = lanemask_lt();
   unsigned total = 0;
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
-    const bool c = L.ok(j) && key[j] >= tau;
+    const bool c = L.ok(j) && (tau == 0u || v[j] >= tau_v);
     const unsigned b = __ballot_sync(kFull, c);
     const unsigned pos = total + __popc(b & below);
     if (c && pos < 32) {
-      s_ck[pos] = key[j];
+      s_cv[pos] = v[j];
       s_ce[pos] = lane + 32 * j;
     }
     total += __popc(b);
   }
 
   my_e = 0;
-  uint32_t my_k = 0;
+  float my_v = 0.0f;
   if (total <= 32) {
-    // zero keys pad the candidates to a multiple of 4: they beat no candidate
-    if (lane >= (int)total && lane < (int)((total + 3) & ~3u)) s_ck[lane] = 0u;
+    // -inf pads the candidates to a multiple of 4: a pad beats no candidate
+    if (lane >= (int)total && lane < (int)((total + 3) & ~3u)) s_cv[lane] = kNoCand;
     __syncwarp();
-    const uint32_t ck = lane < (int)total ? s_ck[lane] : 0u;
+    const float cv = lane < (int)total ? s_cv[lane] : 0.0f;
     const int ce = lane < (int)total ? s_ce[lane] : 0;
+    // rank = candidates with a larger logit, or an equal one at a lower
+    // position (a lower expert id); -0 and +0 compare equal
     int rank = 0;
     for (int j = 0; j < (int)total; j += 4) {
-      const uint4 q = *reinterpret_cast<const uint4 *>(s_ck + j);  // broadcast
-      rank += (q.x > ck || (q.x == ck && j < lane)) ? 1 : 0;
-      rank += (q.y > ck || (q.y == ck && j + 1 < lane)) ? 1 : 0;
-      rank += (q.z > ck || (q.z == ck && j + 2 < lane)) ? 1 : 0;
-      rank += (q.w > ck || (q.w == ck && j + 3 < lane)) ? 1 : 0;
+      const float4 q = *reinterpret_cast<const float4 *>(s_cv + j);  // broadcast
+      rank += (q.x > cv || (q.x == cv && j < lane)) ? 1 : 0;
+      rank += (q.y > cv || (q.y == cv && j + 1 < lane)) ? 1 : 0;
+      rank += (q.z > cv || (q.z == cv && j + 2 < lane)) ? 1 : 0;
+      rank += (q.w > cv || (q.w == cv && j + 3 < lane)) ? 1 : 0;
     }
     __syncwarp();
     if (lane < (int)total && rank < k) {
-      s_ck[rank] = ck;
+      s_cv[rank] = cv;
       s_ce[rank] = ce;
     }
     __syncwarp();
     if (lane < k) {
-      my_k = s_ck[lane];
+      my_v = s_cv[lane];
       my_e = s_ce[lane];
     }
     __syncwarp();
   } else {
     // many ties at tau: scan every element each round
     for (int r = 0; r < k; ++r) {
-      uint32_t bk = 0;
+      float bf = kNoCand;
       int be = 0x7fffffff;
 #pragma unroll
       for (int j = 0; j < EPL; ++j)
-        if (key[j] > bk) {  // strict: the lowest slot wins ties
-          bk = key[j];
+        if (v[j] > bf) {  // strict: the lowest slot wins ties
+          bf = v[j];
           be = lane + 32 * j;
         }
+      const uint32_t bk = be != 0x7fffffff ? order_key(bf) : 0u;
       const uint32_t kmx = __reduce_max_sync(kFull, bk);
       const int ewin = (int)__reduce_min_sync(kFull, (bk == kmx) ? (unsigned)be : 0x7fffffffu);
       if (lane == (ewin & 31)) {
 #pragma unroll
         for (int j = 0; j < EPL; ++j)
-          if (j == (ewin >> 5)) key[j] = 0;
+          if (j == (ewin >> 5)) v[j] = kNoCand;
       }
       if (lane == r) {
         my_e = ewin;
-        my_k = kmx;
+        my_v = key_value(kmx);
       }
     }
   }
   // gate weights, one per lane: softmax probability of the pick
-  my_w = (lane < k) ? expf(key_value(my_k) - m) / s : 0.0f;
+  my_w = (lane < k) ? expf(my_v - m) / s : 0.0f;
   if (renorm) {
     const float tot = warp_sum(lane < k ? my_w : 0.0f);
     my_w = my_w / tot;

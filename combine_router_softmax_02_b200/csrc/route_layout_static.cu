@@ -34,7 +34,7 @@ template <int EPL, bool FULL, int KM>
 __global__ void __launch_bounds__(kTile) route_layout_kernel(RouteArgs ra, LayoutArgs a, DeviceCtx ctx) {
   extern __shared__ int4 smem_raw[];
   int *sm = reinterpret_cast<int *>(smem_raw);
-  __shared__ __align__(16) uint32_t s_ck[kWarps][32];
+  __shared__ __align__(16) float s_cv[kWarps][32];
   __shared__ int s_ce[kWarps][32];
   __shared__ int s_flag;
   const SmemPlan P = layout::smem_plan(a.E, a.NBp, a.R, true);
@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kTile) route_layout_kernel(RouteArgs ra, Layou
     int e;
     float w;
     route::route_token<EPL, FULL>(ra.logits + (size_t)t * a.E, a.E, a.k, ra.n_groups, ra.gpt,
-                                  ra.renorm, L, s_ck[warp], s_ce[warp], lane, e, w, bad);
+                                  ra.renorm, L, s_cv[warp], s_ce[warp], lane, e, w, bad);
     int r = -1;
     if (lane < a.k) {
       ra.idx_out[(size_t)t * a.k + lane] = e;

@@ -9,7 +9,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          int E, int k, int n_groups, int gpt,
                                                          int renorm, int *__restrict__ idx_out,
                                                          float *__restrict__ w_out, DeviceCtx ctx) {
-  __shared__ __align__(16) uint32_t s_ck[8][32];  // per-warp candidate keys
+  __shared__ __align__(16) float s_cv[8][32];  // per-warp candidate logits
   __shared__ int s_ce[8][32];       // and their experts
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     int my_e;
     float my_w;
     bool bad = false;
-    route::route_token<EPL, FULL>(logits + (size_t)t * E, E, k, n_groups, gpt, renorm, L, s_ck[warp],
+    route::route_token<EPL, FULL>(logits + (size_t)t * E, E, k, n_groups, gpt, renorm, L, s_cv[warp],
                             s_ce[warp], lane, my_e, my_w, bad);
     if (__any_sync(route::kFull, bad) && lane == 0) set_status(ctx.status, MOE_ERR_BAD_INPUT);
     if (lane < k) {
