@@ -306,14 +306,25 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
     reinterpret_cast<int4 *>(s_ppre + q * a.NBp)[v] = pre;
   }
   __syncthreads();
-  for (int b = tid; b < a.NB; b += kTile) {
+  // the Q partial rows summed per bin: G threads per bin (a power of two <= 32
+  // that divides the warp), each over every G-th row, then a shuffle tree
+  const int G = a.NB >= kTile ? 1 : min(32, 1 << (31 - __clz(kTile / a.NB)));
+  for (int b0 = 0; b0 < a.NB; b0 += kTile / G) {  // uniform trip count over the block
+    const int b = b0 + tid / G, sub = tid % G;
     int tot = 0, pre = 0;
-    for (int q = 0; q < Q; ++q) {
-      tot += s_ptot[q * a.NBp + b];
-      pre += s_ppre[q * a.NBp + b];
+    if (b < a.NB)
+      for (int q = sub; q < Q; q += G) {
+        tot += s_ptot[q * a.NBp + b];
+        pre += s_ppre[q * a.NBp + b];
+      }
+    for (int d = G >> 1; d > 0; d >>= 1) {
+      tot += __shfl_down_sync(kFull, tot, d, G);
+      pre += __shfl_down_sync(kFull, pre, d, G);
     }
-    s_cnt[b] = tot;
-    s_base[b] = pre;
+    if (b < a.NB && sub == 0) {
+      s_cnt[b] = tot;
+      s_base[b] = pre;
+    }
   }
   __syncthreads();
 

@@ -11,10 +11,11 @@ __global__ void __launch_bounds__(256) replica_assign_kernel(
     const int *__restrict__ slots, int n_entries, const int *__restrict__ slot_rank, int S, int R,
     int *__restrict__ expert_slot, int *__restrict__ expert_rank, int *__restrict__ rank_active,
     DeviceCtx ctx) {
-  extern __shared__ int sm[];
+  extern __shared__ int4 sm_raw[];  // 16-byte aligned
+  int *sm = reinterpret_cast<int *>(sm_raw);
   const MetroPlan P = metro_plan(E, n_entries, R);
-  metro_stage(E, off, slots, n_entries, slot_rank, S, R, sm, P);
-  metro_solve(counts, E, R, sm, P, sm + P.total, true, expert_slot, expert_rank, rank_active, ctx);
+  metro_stage(E, off, slots, n_entries, slot_rank, S, R, counts, sm, P);
+  metro_solve(nullptr, E, R, sm, P, sm + P.total, true, expert_slot, expert_rank, rank_active, ctx);
 }
 
 }  // namespace

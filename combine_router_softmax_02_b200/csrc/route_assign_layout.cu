@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kTile) route_assign_layout_kernel(FrontArgs f,
   for (int i = tid; i < a.E; i += kTile)
     if (s_hist[i]) atomicAdd(&a.cnt[i], s_hist[i]);
   __syncthreads();  // s_hist is read out before the replica map reuses its memory
-  metro_stage(a.E, f.off, f.slots, f.n_entries, f.slot_rank, f.S, a.R, smm, M);
+  metro_stage(a.E, f.off, f.slots, f.n_entries, f.slot_rank, f.S, a.R, nullptr, smm, M);
   if (!layout::grid_barrier(a, ctx, &s_flag, 1)) return;
 
   // B: the greedy in every block, straight into the layout's expert -> rank map
