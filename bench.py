@@ -77,73 +77,113 @@ def ncu_traffic(kernel: str, workload: str):
     return int(t.group(1))
 
 
+_SAMPLER = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+uuid, period = sys.argv[1], float(sys.argv[2])
+try:
+    h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+except pynvml.NVMLError:
+    h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[3]))
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    t = time.perf_counter()
+    print(t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+          pynvml.nvmlDeviceGetCurrentClocksEventReasons(h), pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0,
+          flush=True)
+    time.sleep(period)
+"""
+
+
+class ClockRecord:
+    """A clock record to fill in once the sampler has stopped: the host-time
+    windows of one timed region (or several)."""
+
+    def __init__(self, regions):
+        self.regions = regions
+
+
+def fill_clock_records(obj, sampler):
+    """Replaces every ClockRecord in a nested dict/list by its statistics."""
+    if isinstance(obj, ClockRecord):
+        return sampler.stats(obj.regions)
+    if isinstance(obj, dict):
+        return {k: fill_clock_records(v, sampler) for k, v in obj.items()}
+    if isinstance(obj, list):
+        return [fill_clock_records(v, sampler) for v in obj]
+    return obj
+
+
 class ClockSampler:
     """SM clock, power and clock-event reasons of the GPU, read through NVML
-    every 10 ms in a background thread (reading only; no setting is touched).
-    ``stats(regions)`` summarises the samples taken inside the given host-time
-    windows, so each timed region gets its own record."""
+    every 10 ms by a separate process (reading only; no setting is touched),
+    so that sampling takes no time from the process that launches the
+    kernels.  Samples carry time.perf_counter() stamps (CLOCK_MONOTONIC, the
+    same clock in both processes); ``stats(regions)`` summarises the samples
+    taken inside the given host-time windows, so each timed region gets its
+    own record."""
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
                ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
     def __init__(self, dev, period_s: float = 0.01):
         self.dev, self.period = dev, period_s
-        self.samples = []          # (host time, sm MHz, reasons bitmask, power W)
+        self.proc = None
+        self.samples = None        # (host time, sm MHz, reasons bitmask, power W), filled by stop()
         self.sm_max = None
         self.error = None
-        self._stop = None
-        self._thread = None
-
-    def _handle(self):
-        import pynvml
-        import torch
-        pynvml.nvmlInit()
-        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
-        try:
-            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
-        except pynvml.NVMLError:
-            return pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
 
     def start(self):
-        import threading
+        import torch
+        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        index = self.dev.index if self.dev.index is not None else 0
+        if "CUDA_VISIBLE_DEVICES" in os.environ:
+            vis = os.environ["CUDA_VISIBLE_DEVICES"].split(",")
+            index = int(vis[index]) if index < len(vis) and vis[index].strip().isdigit() else index
+        import subprocess
         try:
-            import pynvml
-            h = self._handle()
-            self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
-        except Exception as e:  # no NVML: the record says so
-            self.error = f"NVML unavailable: {e}"
-            return
-        self._stop = threading.Event()
-
-        def loop():
-            while not self._stop.is_set():
-                try:
-                    t = time.perf_counter()
-                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
-                    self.samples.append((t, float(sm), int(rs), pw))
-                except Exception as e:
-                    self.error = str(e)
-                self._stop.wait(self.period)
-
-        self._thread = threading.Thread(target=loop, daemon=True)
-        self._thread.start()
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER, uuid, str(self.period), str(index)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        except Exception as e:  # no sampler: the record says so
+            self.error = f"clock sampler unavailable: {e}"
+        time.sleep(0.5)  # the sampler is running before the first timed region
 
     def stop(self):
-        if self._thread is not None:
-            self._stop.set()
-            self._thread.join(timeout=5)
+        if self.samples is not None:
+            return
+        self.samples = []
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, err = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, err = self.proc.communicate()
+        for line in out.splitlines():
+            parts = line.split()
+            try:
+                if parts[0] == "max":
+                    self.sm_max = float(parts[1])
+                else:
+                    self.samples.append((float(parts[0]), float(parts[1]), int(parts[2]), float(parts[3])))
+            except (ValueError, IndexError):
+                continue
+        if not self.samples and self.error is None:
+            self.error = "NVML sampler gave no samples: " + " ".join(err.split())[:200]
 
     def stats(self, regions):
-        if self.error and not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [self.error], "samples": 0}
-        sel = [x for x in list(self.samples) if any(a <= x[0] <= b for a, b in regions)]
+        self.stop()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [self.error or "no samples"],
+                    "samples": 0}
+        sel = [x for x in self.samples if any(a <= x[0] <= b for a, b in regions)]
         reasons = sorted({n for x in sel for n, bit in self.REASONS if x[2] & bit})
         sm = [x[1] for x in sel]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_mhz_min": min(sm) if sm else None,
                 "sm_max_mhz": self.sm_max, "reasons": reasons, "samples": len(sel),
                 "power_w_max": max(x[3] for x in sel) if sel else None,
-                "seconds": round(sum(b - a for a, b in regions), 3), "source": "NVML, 10 ms"}
+                "seconds": round(sum(b - a for a, b in regions), 3), "source": "NVML, 10 ms, sampler process"}
 
 
 # ---------------------------------------------------------- byte accounting
@@ -436,7 +476,7 @@ def measure_extra(moe, label, cfg, fused, graph, e2e, args, dev, stream, barrier
                   "unit": "token-rows/s", "kernels_us": per,
                   "kernels_GBps": {n: bytes_[n] / (per[n] * 1e-6) / 1e9 for n in per},
                   "hbm_GBps": step_total / (ms / steps * 1e-3) / 1e9,
-                  "gpu_launches": int(launches), "clocks": sampler.stats(regions[-1:])},
+                  "gpu_launches": int(launches), "clocks": ClockRecord(regions[-1:])},
         "roofline": kernel_rooflines(cfg, per, bytes_, peak),
         "l2": l2_note(cfg, rows),
     }
@@ -446,14 +486,14 @@ def measure_extra(moe, label, cfg, fused, graph, e2e, args, dev, stream, barrier
         check_status(moe, f"after graph replays of {label}")
         entry["cuda_graph"] = {"steps": gsteps, "ms_per_step": gms / gsteps, "us_per_step": gms / gsteps * 1e3,
                                "value": rows * gsteps / (gms * 1e-3), "unit": "token-rows/s",
-                               "kernels_per_step": per_pass, "clocks": sampler.stats(regions[-1:])}
+                               "kernels_per_step": per_pass, "clocks": ClockRecord(regions[-1:])}
     if e2e:
         esteps = max(1, min(args.steps, 10))
         ems, info = timed_e2e(wl, stream, esteps, min(args.warmup, 2), args.e2e_chunks, barrier, regions)
         check_status(moe, f"after the end-to-end leg of {label}")
         entry["e2e"] = {"value": rows * esteps / (ems * 1e-3), "unit": "token-rows/s",
                         "ms_per_step": ems / esteps, **info}
-    entry["clocks"] = sampler.stats(regions)
+    entry["clocks"] = ClockRecord(list(regions))
     del wl
     return entry, regions
 
@@ -544,9 +584,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             extra[label] = entry
             regions += reg
             torch.cuda.empty_cache()
+    sampler.stop()
     clocks_all = sampler.stats(regions)
     clocks_head = sampler.stats(head_regions)
-    sampler.stop()
+    extra = fill_clock_records(extra, sampler)
 
     # whole-job aggregation: max time over ranks, rows summed over ranks
     agg = aggregate(dist, dev, [elapsed_ms, e2e_ms], [rows * args.steps, rows * e2e_steps])

@@ -15,6 +15,8 @@
 // + (rows in earlier lanes of the warp): the stable (token-order) prefix scan.
 // Phase 1 counts every block's rows per bin, a grid barrier publishes the
 // count table, phase 2 scans it and writes the rows (layout_common.cuh).
+// Small token sets in the mask modes take one pass instead: every block counts
+// every token itself, with no count table and no barrier.
 // Ranks and groups (at most 64 each) are 64-bit masks per token, one ballot
 // per bin per warp; experts (PER_PICK, up to 1024 bins) are merged in
 // ascending (rank, expert) order with redux.sync.min.
@@ -35,14 +37,29 @@ __global__ void __launch_bounds__(kTile) layout_kernel(LayoutArgs a, DeviceCtx c
   layout_phases<KM, MODE>(a, P, sm, t0, t1, ctx, &s_flag, 1);
 }
 
-std::atomic<unsigned long long> g_smem_set[4][3];
+// Small token sets in the mask modes: one pass, no count table, no barrier
+// (a kernel of its own, so the two-phase kernel's code stays as it is).
+template <int KM, int MODE>
+__global__ void __launch_bounds__(kTile) layout_one_pass_kernel(LayoutArgs a, DeviceCtx ctx) {
+  extern __shared__ int4 smem_raw[];
+  int *sm = reinterpret_cast<int *>(smem_raw);
+  const SmemPlan P = smem_plan(a.E, a.NBp, a.R, false);
+  const int t0 = blockIdx.x * a.chunk, t1 = min(a.T, t0 + a.chunk);
+  smem_init(a, P, sm);
+  layout_single_pass<KM, MODE>(a, P, sm, t0, t1, ctx);
+}
+
+std::atomic<unsigned long long> g_smem_set[4][3][2];
 
 template <int KM, int MODE>
 cudaError_t launch_k(const LayoutArgs &a0, int kind, const DeviceCtx &ctx, cudaStream_t s) {
   LayoutArgs a = a0;
   const size_t smem = sizeof(int) * (size_t)smem_plan(a.E, a.NBp, a.R, false).total;
+  const bool one = single_pass(a.T, MODE);
   auto kern = layout_kernel<KM, MODE>;
-  cudaError_t err = set_smem_limit_once(kern, 200 * 1024, g_smem_set[kind][MODE]);
+  if constexpr (MODE != MOE_LAYOUT_PER_PICK)
+    if (one) kern = layout_one_pass_kernel<KM, MODE>;
+  cudaError_t err = set_smem_limit_once(kern, 200 * 1024, g_smem_set[kind][MODE][one]);
   if (err != cudaSuccess) return err;
   int resident = 0;
   if ((err = max_resident_blocks((const void *)kern, smem, ctx, resident)) != cudaSuccess) return err;
@@ -51,7 +68,8 @@ cudaError_t launch_k(const LayoutArgs &a0, int kind, const DeviceCtx &ctx, cudaS
   // (28.9 us against 32.1-32.5)
   const int bps = MODE == MOE_LAYOUT_TWO_HOP ? 1 : kBlocksPerSm;
   split_tokens(a.T, resident < bps * ctx.num_sms ? resident : bps * ctx.num_sms, a.nblk, a.chunk);
-  if ((err = cudaMemsetAsync(a.bar, 0, sizeof(int) * 16, s)) != cudaSuccess) return err;
+  if (!one)  // the barrier words start at zero
+    if ((err = cudaMemsetAsync(a.bar, 0, sizeof(int) * 16, s)) != cudaSuccess) return err;
   void *args[] = {&a, const_cast<DeviceCtx *>(&ctx)};
   err = cudaLaunchCooperativeKernel((const void *)kern, dim3(a.nblk), dim3(kTile), args, smem, s);
   if (err != cudaSuccess) return err;

@@ -282,10 +282,8 @@ __device__ __forceinline__ bool grid_barrier(const LayoutArgs &a, const DeviceCt
 
 // ------------------------------------------------------------- phase 2 ----
 // Per-bin totals (into s_cnt) and this block's base (into s_base) from the
-// count table, then the segment offsets; block 0 writes the layout's offsets.
-template <int MODE>
-__device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const SmemPlan &P, int *sm,
-                                                  DeviceCtx ctx) {
+// count table.
+__device__ __forceinline__ void gather_counts(const LayoutArgs &a, const SmemPlan &P, int *sm) {
   const int tid = threadIdx.x;
   const int V = a.NBp / 4;                      // 16-byte vectors per table row
   const int Q = V >= kTile ? 1 : kTile / V;     // row groups
@@ -306,9 +304,10 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
     reinterpret_cast<int4 *>(s_ppre + q * a.NBp)[v] = pre;
   }
   __syncthreads();
-  // the Q partial rows summed per bin: G threads per bin (a power of two <= 32
-  // that divides the warp), each over every G-th row, then a shuffle tree
-  const int G = a.NB >= kTile ? 1 : min(32, 1 << (31 - __clz(kTile / a.NB)));
+  // the Q partial rows summed per bin: with few bins (Q >= 32 partial rows) G
+  // threads per bin (a power of two <= 32), each over every G-th row, then a
+  // shuffle tree; with many bins one thread per bin
+  const int G = a.NB > 32 ? 1 : min(32, 1 << (31 - __clz(kTile / a.NB)));
   for (int b0 = 0; b0 < a.NB; b0 += kTile / G) {  // uniform trip count over the block
     const int b = b0 + tid / G, sub = tid % G;
     int tot = 0, pre = 0;
@@ -327,6 +326,16 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
     }
   }
   __syncthreads();
+}
+
+// Segment offsets from the per-bin totals (s_cnt); every bin's running base
+// (s_base, the rows of the bin before this block) moves past them.  Block 0
+// writes the layout's offsets and row counts.
+template <int MODE>
+__device__ __forceinline__ void segment_offsets(const LayoutArgs &a, const SmemPlan &P, int *sm,
+                                                DeviceCtx ctx) {
+  const int tid = threadIdx.x, blk = blockIdx.x;
+  int *s_cnt = sm + P.cnt, *s_base = sm + P.base;
 
   // segment offsets
   int *s_seg = sm + P.seg;
@@ -416,9 +425,27 @@ __device__ __forceinline__ void bases_from_counts(const LayoutArgs &a, const Sme
   __syncthreads();
 }
 
+// Adds one tile's rows to the block's send-count matrix: source rank of the
+// token -> its ranks (lane i holds the warp's ballots of ranks i, i + 32).
+__device__ __forceinline__ void add_send_counts(const LayoutArgs &a, const SmemPlan &P, int *sm,
+                                                unsigned long long dmask, const Ballots &bl, int t,
+                                                bool live) {
+  const int lane = threadIdx.x & 31;
+  int *s_send = sm + P.send;
+  const int src = live ? t / a.tpr : 0;
+  const int src0 = __shfl_sync(kFull, src, 0);
+  if (__all_sync(kFull, !live || src == src0)) {
+    if (bl.b0) atomicAdd(&s_send[src0 * a.R + lane], __popc(bl.b0));
+    if (bl.b1) atomicAdd(&s_send[src0 * a.R + lane + 32], __popc(bl.b1));
+  } else {
+    for (unsigned long long m = dmask; m; m &= m - 1)
+      atomicAdd(&s_send[src * a.R + __ffsll((long long)m) - 1], 1);
+  }
+}
+
 // Rows of one tile of mask-bin tokens (DEDUP, TWO_HOP).  Every thread of the
 // block calls it; `t` is the thread's token, `live` whether it has one.
-template <int KM, int MODE>
+template <int KM, int MODE, bool SEND>
 __device__ __forceinline__ void rows_mask_tile(const LayoutArgs &a, const SmemPlan &P, int *sm,
                                                const TokenPicks<KM> &p, const Ballots &bl, int t,
                                                bool live, bool &over) {
@@ -432,17 +459,7 @@ __device__ __forceinline__ void rows_mask_tile(const LayoutArgs &a, const SmemPl
     if (lane < a.G) s_w[a.R + lane] = bl.g0;
     if (lane + 32 < a.G) s_w[a.R + lane + 32] = bl.g1;
   }
-  // send counts: source rank of the token -> its ranks
-  int *s_send = sm + P.send;
-  const int src = live ? t / a.tpr : 0;
-  const int src0 = __shfl_sync(kFull, src, 0);
-  if (__all_sync(kFull, !live || src == src0)) {
-    if (b0) atomicAdd(&s_send[src0 * a.R + lane], __popc(b0));
-    if (b1) atomicAdd(&s_send[src0 * a.R + lane + 32], __popc(b1));
-  } else {
-    for (unsigned long long m = p.dmask; m; m &= m - 1)
-      atomicAdd(&s_send[src * a.R + __ffsll((long long)m) - 1], 1);
-  }
+  if (SEND) add_send_counts(a, P, sm, p.dmask, bl, t, live);
   __syncthreads();
   int *s_base = sm + P.base;
   for (int b = tid; b < a.NB; b += kTile) {
@@ -570,11 +587,10 @@ __device__ __forceinline__ void rows_pick_tile(const LayoutArgs &a, const SmemPl
 // and `pre_bl`: the thread's picks (with weights) and its warp's ballots kept
 // from phase 1 when the chunk is one tile, else null (loaded again, tile by
 // tile).
-template <int KM, int MODE>
-__device__ __forceinline__ void phase2(const LayoutArgs &a, const SmemPlan &P, int *sm, int t0,
-                                       int t1, DeviceCtx ctx, const TokenPicks<KM> *pre,
-                                       const Ballots *pre_bl) {
-  bases_from_counts<MODE>(a, P, sm, ctx);
+template <int KM, int MODE, bool SEND>
+__device__ __forceinline__ void rows_loop(const LayoutArgs &a, const SmemPlan &P, int *sm, int t0,
+                                          int t1, DeviceCtx ctx, const TokenPicks<KM> *pre,
+                                          const Ballots *pre_bl) {
   bool over = false, bad = false;
   const int lane = threadIdx.x & 31;
   for (int base = t0; base < t1; base += kTile) {
@@ -589,14 +605,24 @@ __device__ __forceinline__ void phase2(const LayoutArgs &a, const SmemPlan &P, i
       rows_pick_tile<KM>(a, P, sm, p, t, live, over);
     } else {
       const Ballots bl = pre_bl ? *pre_bl : mask_ballots<MODE>(a, p.dmask, p.gmask, live, lane);
-      rows_mask_tile<KM, MODE>(a, P, sm, p, bl, t, live, over);
+      rows_mask_tile<KM, MODE, SEND>(a, P, sm, p, bl, t, live, over);
     }
   }
   if (over) set_status(ctx.status, MOE_ERR_CAPACITY);
-  // the block's send counts (send_counts was cleared before the barrier)
-  const int *s_send = sm + P.send;
-  for (int i = threadIdx.x; i < a.R * a.R; i += kTile)
-    if (s_send[i]) atomicAdd(&a.L.send_counts[i], s_send[i]);
+  if (SEND) {  // the block's send counts (send_counts was cleared before the barrier)
+    const int *s_send = sm + P.send;
+    for (int i = threadIdx.x; i < a.R * a.R; i += kTile)
+      if (s_send[i]) atomicAdd(&a.L.send_counts[i], s_send[i]);
+  }
+}
+
+template <int KM, int MODE>
+__device__ __forceinline__ void phase2(const LayoutArgs &a, const SmemPlan &P, int *sm, int t0,
+                                       int t1, DeviceCtx ctx, const TokenPicks<KM> *pre,
+                                       const Ballots *pre_bl) {
+  gather_counts(a, P, sm);
+  segment_offsets<MODE>(a, P, sm, ctx);
+  rows_loop<KM, MODE, true>(a, P, sm, t0, t1, ctx, pre, pre_bl);
 }
 
 // Phase-1 epilogue: the block's counts into its table row; block 0 clears the
@@ -644,6 +670,88 @@ __device__ __forceinline__ bool layout_phases(const LayoutArgs &a, const SmemPla
   if (!grid_barrier(a, ctx, s_flag, round)) return false;
   phase2<KM, MODE>(a, P, sm, t0, t1, ctx, one_tile ? &p : nullptr, one_tile ? &bl : nullptr);
   return true;
+}
+
+// ------------------------------------------------------------ one pass ----
+// Small token sets (mask modes) skip the count table and its grid barrier:
+// every block counts every token's rows per bin itself -- the bin totals and
+// the rows before its own chunk -- and block 0 also counts the whole
+// send-count matrix, walking the tokens in tiles of 256 with the next tile's
+// picks loaded while this one is counted.  A tile costs each block about as
+// much as the barrier and the count-table pass it replaces take in all
+// (clock-stamped on the decode workloads: ~2.5k cycles a tile, against ~4.7 us
+// for the two-phase route at 1024 tokens), so only one or two tiles go this way.
+constexpr int kOnePassTokens = 2 * kTile;
+
+// Whether a layout of T tokens takes the one-pass route.
+__host__ __device__ inline bool single_pass(int T, int mode) {
+  return mode != MOE_LAYOUT_PER_PICK && T <= kOnePassTokens;
+}
+
+// The layout over the block's chunk [t0, t1) in one pass (mask modes), after
+// smem_init; the expert -> rank map is in shared memory.
+template <int KM, int MODE>
+__device__ __forceinline__ void layout_single_pass(const LayoutArgs &a, const SmemPlan &P, int *sm,
+                                                   int t0, int t1, DeviceCtx ctx) {
+  static_assert(MODE != MOE_LAYOUT_PER_PICK, "mask modes only");
+  const int lane = threadIdx.x & 31;
+  int *s_cnt = sm + P.cnt, *s_base = sm + P.base;
+  const int *s_er = sm + P.er;
+  for (int b = threadIdx.x; b < a.NBp; b += kTile) s_base[b] = 0;
+  __syncthreads();
+  auto fetch = [&](int t, int (&e)[KM]) {
+#pragma unroll
+    for (int j = 0; j < KM; ++j) e[j] = (j < a.k && t < a.T) ? a.idx[(size_t)t * a.k + j] : 0;
+  };
+  int nxt[KM];
+  fetch((int)threadIdx.x, nxt);
+  bool bad = false;
+  int c[4] = {0, 0, 0, 0}, cp[4] = {0, 0, 0, 0};
+#pragma unroll 1
+  for (int base = 0; base < a.T; base += kTile) {
+    int e[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) e[j] = nxt[j];
+    fetch(base + kTile + (int)threadIdx.x, nxt);  // the next tile, in flight meanwhile
+    const int t = base + (int)threadIdx.x;
+    const bool live = t < a.T;
+    unsigned long long dmask = 0, gmask = 0;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if (j < a.k && live) {
+        const int ex = e[j];
+        const int r = (unsigned)ex < (unsigned)a.E ? s_er[ex] : -1;
+        if ((unsigned)r < (unsigned)a.R) {
+          dmask |= 1ull << r;
+          gmask |= 1ull << (r / a.rpg);
+        } else {
+          bad = true;
+        }
+      }
+    }
+    const Ballots bl = mask_ballots<MODE>(a, dmask, gmask, live, lane);
+    const unsigned before = __ballot_sync(kFull, live && t < t0);
+    c[0] += __popc(bl.b0);
+    c[1] += __popc(bl.b1);
+    c[2] += __popc(bl.g0);
+    c[3] += __popc(bl.g1);
+    cp[0] += __popc(bl.b0 & before);
+    cp[1] += __popc(bl.b1 & before);
+    cp[2] += __popc(bl.g0 & before);
+    cp[3] += __popc(bl.g1 & before);
+    if (blockIdx.x == 0) add_send_counts(a, P, sm, dmask, bl, t, live);
+  }
+  flush_counts<MODE>(a, lane, s_cnt, c);
+  flush_counts<MODE>(a, lane, s_base, cp);
+  if (bad) set_status(ctx.status, MOE_ERR_BAD_INPUT);
+  __syncthreads();
+  segment_offsets<MODE>(a, P, sm, ctx);
+  rows_loop<KM, MODE, false>(a, P, sm, t0, t1, ctx, nullptr, nullptr);
+  if (blockIdx.x == 0) {
+    __syncthreads();
+    const int *s_send = sm + P.send;
+    for (int i = threadIdx.x; i < a.R * a.R; i += kTile) a.L.send_counts[i] = s_send[i];
+  }
 }
 
 // ---------------------------------------------------------------- host ----

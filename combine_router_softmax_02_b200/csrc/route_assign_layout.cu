@@ -12,7 +12,9 @@
 //      the same expert -> rank map and no block waits for another); block 0
 //      writes expert_slot, expert_rank, rank_active and counts; then every
 //      block counts its chunk's layout bins with that map;
-//   C. after the layout's barrier every block writes its rows (layout_common.cuh).
+//   C. after the layout's barrier every block writes its rows (layout_common.cuh);
+//      small token sets (mask modes) skip that barrier: every block counts every
+//      token's rows itself and writes its own.
 // Every output equals that of moe_route_topk, moe_demand_hist,
 // moe_replica_assign and moe_build_layout called one after the other.
 #include "assign_common.cuh"
@@ -95,12 +97,20 @@ __global__ void __launch_bounds__(kTile) route_assign_layout_kernel(FrontArgs f,
 
   // B + C: the layout with the assigned ranks
   layout::smem_init(a, P, sm, false);
-  if (a.mode == MOE_LAYOUT_DEDUP)
-    layout::layout_phases<KM, MOE_LAYOUT_DEDUP>(a, P, sm, t0, t1, ctx, &s_flag, 2);
-  else if (a.mode == MOE_LAYOUT_TWO_HOP)
-    layout::layout_phases<KM, MOE_LAYOUT_TWO_HOP>(a, P, sm, t0, t1, ctx, &s_flag, 2);
-  else
+  const bool one = layout::single_pass(a.T, a.mode);
+  if (a.mode == MOE_LAYOUT_DEDUP) {
+    if (one)
+      layout::layout_single_pass<KM, MOE_LAYOUT_DEDUP>(a, P, sm, t0, t1, ctx);
+    else
+      layout::layout_phases<KM, MOE_LAYOUT_DEDUP>(a, P, sm, t0, t1, ctx, &s_flag, 2);
+  } else if (a.mode == MOE_LAYOUT_TWO_HOP) {
+    if (one)
+      layout::layout_single_pass<KM, MOE_LAYOUT_TWO_HOP>(a, P, sm, t0, t1, ctx);
+    else
+      layout::layout_phases<KM, MOE_LAYOUT_TWO_HOP>(a, P, sm, t0, t1, ctx, &s_flag, 2);
+  } else {
     layout::layout_phases<KM, MOE_LAYOUT_PER_PICK>(a, P, sm, t0, t1, ctx, &s_flag, 2);
+  }
 }
 
 std::atomic<unsigned long long> g_smem_set[6][2][2];

@@ -72,6 +72,10 @@ def test_layout_multi_tile_chunks(moe, mode, R, rpg):
     (999, 64, 5, 16, 63, W.TWO_HOP, 16, False),    # one group
     (700, 40, 7, 12, 59, W.TWO_HOP, 1, False),     # one rank per group
     (5000, 256, 8, 64, 79, W.TWO_HOP, 4, False),
+    (512, 64, 4, 32, 16, W.DEDUP, 1, True),        # the largest set counted in one pass
+    (513, 64, 4, 32, 17, W.DEDUP, 1, True),        # the smallest one with the count table
+    (512, 128, 8, 64, 8, W.TWO_HOP, 8, False),
+    (513, 128, 8, 64, 9, W.TWO_HOP, 8, False),
 ])
 def test_layout_edges(moe, T, E, k, R, tpr, mode, rpg, skew):
     rng = np.random.default_rng(T + 31 * E + k)
@@ -125,10 +129,12 @@ def test_layout_bad_expert_id(moe):
 
 
 def test_layout_bounded_wait_reports_timeout(moe):
-    """A scan tile that never publishes: its successors' waits run out after
-    the set limit and report MOE_ERR_TIMEOUT; the context stays usable."""
+    """A block that never arrives at the grid barrier: the others' waits run
+    out after the set limit and report MOE_ERR_TIMEOUT; the context stays
+    usable.  6144 tokens: above the size that the layout counts in one pass
+    without a barrier (512), so the barrier path runs."""
     rng = np.random.default_rng(9)
-    T, E, k, R = 256 * 6, 16, 2, 4
+    T, E, k, R = 256 * 24, 16, 2, 4
     idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
     w = np.ones((T, k), np.float32)
     er = (np.arange(E) % R).astype(np.int32)
