@@ -139,6 +139,80 @@ __device__ __forceinline__ void metro_stage(int E, const int *__restrict__ off,
   __syncthreads();
 }
 
+// The replica map loaded into registers before the caller's other work
+// (the fused front end issues these loads before it routes, so their latency
+// hides behind the routing): thread i holds entries i and i + 256 of the
+// offsets, the slot list and the slot -> rank table.  `ok` says the map is
+// small enough (E + 1, entries and slots each <= 512) -- otherwise
+// metro_stage loads it itself.
+struct MetroPrefetch {
+  static constexpr int kPer = 2;
+  bool ok;
+  int off[kPer], slot[kPer], srank[kPer];
+  __device__ __forceinline__ void load(int E, const int *__restrict__ off_g, const int *__restrict__ slots_g,
+                                       int n_entries, const int *__restrict__ slot_rank_g, int S) {
+    ok = E + 1 <= kPer * 256 && n_entries <= kPer * 256 && S <= kPer * 256 && blockDim.x == 256;
+    if (!ok) return;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int i = (int)threadIdx.x + q * 256;
+      off[q] = i <= E ? off_g[i] : 0;
+      slot[q] = i < n_entries ? slots_g[i] : 0;
+      srank[q] = i < S ? slot_rank_g[i] : 0;
+    }
+  }
+};
+
+// metro_stage from a prefetched map (no global loads): the slot -> rank
+// table goes through the P.kw area (free until the solve).
+__device__ __forceinline__ void metro_stage_prefetched(int E, int n_entries, int S, int R,
+                                                       const MetroPrefetch &pf, int *sm,
+                                                       const MetroPlan &P) {
+  int *s_off = sm + P.off, *s_key = sm + P.key, *s_fk = sm + P.fk, *s_srank = sm + P.kw;
+  const int C = (E + 31) / 32;
+#pragma unroll
+  for (int q = 0; q < MetroPrefetch::kPer; ++q) {
+    const int i = (int)threadIdx.x + q * 256;
+    if (i <= E) s_off[i] = pf.off[q];
+    if (i < S) s_srank[i] = pf.srank[q];
+  }
+  for (int i = threadIdx.x; i < C * R; i += blockDim.x) sm[P.mask + i] = 0;
+  for (int i = threadIdx.x; i < R; i += blockDim.x) sm[P.chosen + i] = 0;
+  if (threadIdx.x == 0) sm[P.maxrep] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < MetroPrefetch::kPer; ++q) {
+    const int i = (int)threadIdx.x + q * 256;
+    if (i < n_entries) {
+      const int sl = pf.slot[q];
+      int key = -1;
+      if ((unsigned)sl < (unsigned)S) {
+        const int r = s_srank[sl];
+        if ((unsigned)r < (unsigned)R) key = (r << 15) | sl;
+      }
+      s_key[i] = key;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int lo = s_off[e], hi = s_off[e + 1];
+    int fk = kNone;
+    if (lo < 0 || hi > n_entries || lo > hi) {
+      fk = kBadOff;
+    } else {
+      int nvalid = 0;
+      for (int i = lo; i < hi && nvalid < 2; ++i)
+        if (s_key[i] >= 0) {
+          ++nvalid;
+          fk = s_key[i];
+        }
+      if (nvalid >= 2) fk = kChoice;
+    }
+    s_fk[e] = fk;
+  }
+  __syncthreads();
+}
+
 // The walk by one thread: chosen(r) is byte r % 8 of c[r / 8] (counts stay
 // below 256: at most 255 choice experts), selected and bumped with register
 // operations only; each expert's keys are one 16-byte shared load, issued an

@@ -136,6 +136,7 @@ __device__ __forceinline__ void cp_async_wait() {
 template <typename Tin, typename Tout, int KM>
 __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
     fanin_kernel(FaninArgs a, DeviceCtx ctx) {
+  wait_prior_grids();
   constexpr int VE = Elem<Tin>::kPerVec;
   extern __shared__ uint4 s_stage[];  // [warp][stage 2][KM][32 lanes]
   __shared__ __align__(16) SrcEntry s_tab[kFaninWarps][KM];
@@ -250,6 +251,7 @@ struct TwoHopArgs {
 template <typename Tin, typename Tout, int KM>
 __global__ void __launch_bounds__(kFaninWarps * 32, KM <= 8 ? 3 : 1)
     two_hop_fanin_kernel(TwoHopArgs a, DeviceCtx ctx) {
+  wait_prior_grids();
   constexpr int VE = Elem<Tin>::kPerVec;
   extern __shared__ uint4 s_stage[];  // [warp][stage 2][KM][32 lanes]
   __shared__ __align__(16) SrcEntry s_tab[kFaninWarps][KM];
@@ -348,7 +350,9 @@ cudaError_t launch_two_hop3(const TwoHopArgs &a, const DeviceCtx &ctx, cudaStrea
   static std::atomic<unsigned long long> smem_set{0};
   cudaError_t err = set_smem_limit_once(two_hop_fanin_kernel<Tin, Tout, KM>, smem, smem_set);
   if (err != cudaSuccess) return err;
-  two_hop_fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, smem, s>>>(a, ctx);
+  cudaError_t lerr = launch_after_prior(two_hop_fanin_kernel<Tin, Tout, KM>, dim3((unsigned)blocks),
+                                        dim3(kFaninWarps * 32), (size_t)smem, s, a, ctx);
+  if (lerr != cudaSuccess) return lerr;
   return count_launch(cudaGetLastError());
 }
 
@@ -378,7 +382,9 @@ cudaError_t launch3(const FaninArgs &a, const DeviceCtx &ctx, cudaStream_t s) {
   static std::atomic<unsigned long long> smem_set{0};
   cudaError_t err = set_smem_limit_once(fanin_kernel<Tin, Tout, KM>, smem, smem_set);
   if (err != cudaSuccess) return err;
-  fanin_kernel<Tin, Tout, KM><<<(unsigned)blocks, kFaninWarps * 32, smem, s>>>(a, ctx);
+  cudaError_t lerr = launch_after_prior(fanin_kernel<Tin, Tout, KM>, dim3((unsigned)blocks),
+                                        dim3(kFaninWarps * 32), (size_t)smem, s, a, ctx);
+  if (lerr != cudaSuccess) return lerr;
   return count_launch(cudaGetLastError());
 }
 

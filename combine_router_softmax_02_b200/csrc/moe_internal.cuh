@@ -68,7 +68,33 @@ __device__ __forceinline__ void st_v4(void *p, uint4 v) {
                : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with launch_after_prior()
+// may be scheduled while the kernel before it in the stream is finishing; it
+// waits here, before its first global access, until that kernel has completed
+// and its writes are visible.  Launched any other way, this returns at once.
+__device__ __forceinline__ void wait_prior_grids() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ host ----
+// Launches `kern` so that its blocks may be scheduled before the previous
+// kernel in the stream has completed (the kernel calls wait_prior_grids()
+// before touching memory): the launch latency overlaps the previous kernel's
+// tail.  Captured into a CUDA graph it becomes a programmatic edge.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_after_prior(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                      cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Raises a kernel's dynamic shared-memory limit once per device.
 template <class Kern>
 inline cudaError_t set_smem_limit_once(Kern kern, int bytes, std::atomic<unsigned long long> &done) {

@@ -62,6 +62,7 @@ constexpr int kResidentBlocks = 2;
 
 template <int KM, int NL, int U>
 __global__ void __launch_bounds__(256) fanout_kernel(FanoutArgs a, DeviceCtx ctx) {
+  wait_prior_grids();
   constexpr int W = NL * KM;
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
@@ -118,7 +119,9 @@ cudaError_t launch_kn(const FanoutArgs &a, const DeviceCtx &ctx, cudaStream_t s)
     cudaError_t err = set_smem_limit_once(fanout_kernel<KM, NL, kU>, 160 * 1024, smem_set);
     if (err != cudaSuccess) return err;
   }
-  fanout_kernel<KM, NL, kU><<<(unsigned)blocks, wpb * 32, smem, s>>>(a, ctx);
+  cudaError_t err = launch_after_prior(fanout_kernel<KM, NL, kU>, dim3((unsigned)blocks), dim3(wpb * 32),
+                                       (size_t)smem, s, a, ctx);
+  if (err != cudaSuccess) return err;
   return count_launch(cudaGetLastError());
 }
 

@@ -6,7 +6,8 @@
 // as one cooperative kernel in three phases separated by grid barriers:
 //   A. every block routes the tokens of its chunk (route_common.cuh), adds its
 //      demand histogram into the workspace's demand scratch, and stages the
-//      replica map in shared memory (assign_common.cuh, metro_stage);
+//      replica map in shared memory (assign_common.cuh; a small map's loads
+//      are issued before the routing, so they complete behind it);
 //   B. every block runs the METRO greedy over the complete demand vector into
 //      its own shared memory (the greedy is deterministic, so every block gets
 //      the same expert -> rank map and no block waits for another); block 0
@@ -61,6 +62,8 @@ __global__ void __launch_bounds__(kTile) route_assign_layout_kernel(FrontArgs f,
   const MetroPlan M = metro_plan(a.E, f.n_entries, a.R);
   int *smm = sm + ((a.E + 3) & ~3);  // METRO's scratch (P.er is the first region)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  MetroPrefetch pf;  // the replica map's loads, in flight while the block routes
+  pf.load(a.E, f.off, f.slots, f.n_entries, f.slot_rank, f.S);
   int *s_hist = sm + P.hist;
   for (int i = tid; i < a.E; i += kTile) s_hist[i] = 0;
   __syncthreads();
@@ -86,7 +89,10 @@ __global__ void __launch_bounds__(kTile) route_assign_layout_kernel(FrontArgs f,
   for (int i = tid; i < a.E; i += kTile)
     if (s_hist[i]) atomicAdd(&a.cnt[i], s_hist[i]);
   __syncthreads();  // s_hist is read out before the replica map reuses its memory
-  metro_stage(a.E, f.off, f.slots, f.n_entries, f.slot_rank, f.S, a.R, nullptr, smm, M);
+  if (pf.ok)
+    metro_stage_prefetched(a.E, f.n_entries, f.S, a.R, pf, smm, M);
+  else
+    metro_stage(a.E, f.off, f.slots, f.n_entries, f.slot_rank, f.S, a.R, nullptr, smm, M);
   if (!layout::grid_barrier(a, ctx, &s_flag, 1)) return;
 
   // B: the greedy in every block, straight into the layout's expert -> rank map

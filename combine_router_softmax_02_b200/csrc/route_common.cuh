@@ -45,6 +45,12 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+// e^x computed as 2^(x log2 e) with exp2f (documented within 2 ulp): a
+// multiply and the exponent unit instead of expf's range reduction.  The
+// product's rounding adds |x| units of roundoff to the relative error.
+constexpr float kLog2e = 1.44269504088896341f;
+__device__ __forceinline__ float exp_via_exp2(float x) { return exp2f(x * kLog2e); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(kFull, v, d);
@@ -104,7 +110,7 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
   float s = 0.0f;
 #pragma unroll
   for (int j = 0; j < EPL; ++j)
-    if (L.ok(j)) s += expf(v[j] - m);
+    if (L.ok(j)) s += exp_via_exp2(v[j] - m);
   s = warp_sum(s);
 
   bool fresh = true;  // lm is still the lane maximum (then the warp max is `top`)
@@ -218,7 +224,7 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
     }
   }
   // gate weights, one per lane: softmax probability of the pick
-  my_w = (lane < k) ? expf(my_v - m) / s : 0.0f;
+  my_w = (lane < k) ? exp_via_exp2(my_v - m) / s : 0.0f;
   if (renorm) {
     const float tot = warp_sum(lane < k ? my_w : 0.0f);
     my_w = my_w / tot;

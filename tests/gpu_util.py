@@ -6,10 +6,14 @@ oracle), with u = 2**-24 the float32 unit roundoff:
 
 * gate weight of a pick with logit v, token max m and token minimum lo, when
   E experts are spread over ceil(E/32) slots per lane:
-  |w_dev - w| <= (m - v + m - lo + ceil(E/32) + 12) * u * w.  The subtraction
-  v - m rounds by at most |v - m| u in the exponent's argument, expf adds 2
-  ulp, the sum over experts adds ceil(E/32) + 5 roundings of positive terms
-  plus the worst exponent error of any term, the division one more.
+  |w_dev - w| <= (2.25 (m - v + m - lo) + ceil(E/32) + 14) * u * w.  Each
+  exponential is exp2f(t * log2 e), t = v - m: the subtraction rounds t by a
+  relative u, the float32 log2 e is off by 0.23 u, the product rounds by u,
+  so the argument is off by at most 2.23 |t| u in relative terms, which is
+  2.23 |t| u relative in the result; exp2f adds 2 ulp (<= 4 u).  The
+  numerator's term is 2.23 (m - v) + 4; the sum over experts carries the
+  worst term's 2.23 (m - lo) + 4 plus ceil(E/32) + 5 roundings of positive
+  terms; the division one more.
 * dedup coefficient (sum of a token's weights on a rank, float32 in pick
   order): the largest weight bound plus k u.
 * combine: |out_dev - out| <= 1e-5 * sum_i |c_i y_i| plus one unit in the last
@@ -63,7 +67,7 @@ def weight_tol(logits: np.ndarray, idx: np.ndarray) -> np.ndarray:
     lo = lg.min(axis=1, keepdims=True)
     v = np.take_along_axis(lg, idx.astype(np.int64), axis=1)
     epl = math.ceil(lg.shape[1] / 32)
-    return ((m - v) + (m - lo) + epl + 12) * U
+    return (2.25 * ((m - v) + (m - lo)) + epl + 14) * U
 
 
 def assert_weights(w_dev, w_ref, logits, idx, renormalize=False):
