@@ -366,18 +366,27 @@ def timed_steps(wl: Workload, stream, steps: int, barrier, regions: list, per_ke
     return t0.elapsed_time(t1), per, launches
 
 
-def timed_graph(wl: Workload, stream, steps: int, warmup: int, barrier, regions: list):
+def timed_graph(wl: Workload, stream, steps, warmup: int, barrier, regions: list):
     """The pass captured once in a CUDA graph, replayed `steps` times (no host
-    launch latency between the kernels).  Returns (elapsed ms, kernels per pass)."""
+    launch latency between the kernels); `steps` may be a function of the
+    measured ms per replay (timed over the warm-up replays).  Returns (elapsed
+    ms, kernels per pass, replays)."""
     import torch
     g = torch.cuda.CUDAGraph()
     n0 = wl.moe.kernel_launches()
     with torch.cuda.graph(g):
         wl.step(torch.cuda.current_stream(wl.dev))
     per_pass = wl.moe.kernel_launches() - n0
-    for _ in range(warmup):
+    w0 = torch.cuda.Event(enable_timing=True)
+    w1 = torch.cuda.Event(enable_timing=True)
+    g.replay()
+    w0.record(stream)
+    for _ in range(max(1, warmup - 1)):
         g.replay()
+    w1.record(stream)
     barrier()
+    if callable(steps):
+        steps = steps(w0.elapsed_time(w1) / max(1, warmup - 1))
     g0 = torch.cuda.Event(enable_timing=True)
     g1 = torch.cuda.Event(enable_timing=True)
     h0 = time.perf_counter()
@@ -389,7 +398,7 @@ def timed_graph(wl: Workload, stream, steps: int, warmup: int, barrier, regions:
     regions.append((h0, time.perf_counter()))
     ms = g0.elapsed_time(g1)
     del g
-    return ms, per_pass
+    return ms, per_pass, steps
 
 
 def timed_e2e(wl: Workload, stream, steps: int, warmup: int, chunks: int, barrier, regions: list):
@@ -481,8 +490,8 @@ def measure_extra(moe, label, cfg, fused, graph, e2e, args, dev, stream, barrier
         "l2": l2_note(cfg, rows),
     }
     if graph:
-        gsteps = steps_for(ms_probe, args.min_region_s, args.steps)
-        gms, per_pass = timed_graph(wl, stream, gsteps, args.warmup, barrier, regions)
+        gms, per_pass, gsteps = timed_graph(wl, stream, lambda ms: steps_for(ms, args.min_region_s, args.steps),
+                                            args.warmup, barrier, regions)
         check_status(moe, f"after graph replays of {label}")
         entry["cuda_graph"] = {"steps": gsteps, "ms_per_step": gms / gsteps, "us_per_step": gms / gsteps * 1e3,
                                "value": rows * gsteps / (gms * 1e-3), "unit": "token-rows/s",
@@ -547,7 +556,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     head_regions = list(regions)
     eager_ms = elapsed_ms
     if args.graph:
-        elapsed_ms, per_pass = timed_graph(wl, stream, args.steps, args.warmup, barrier, regions)
+        elapsed_ms, per_pass, _ = timed_graph(wl, stream, args.steps, args.warmup, barrier, regions)
         launches = per_pass * args.steps
         head_regions = regions[-1:]
         check_status(moe, "after graph replays")
