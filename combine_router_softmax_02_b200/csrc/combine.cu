@@ -108,6 +108,12 @@ struct SrcEntry {
 };
 
 constexpr int kFaninWarps = 8;
+// Few output rows (decode) are split into column slices until about this many
+// warps per SM (row_slices): a sweep of 8, 12, 16, 24 and 32 on the 1024-token
+// decode step put combine at 20.5, 20.5, 20.2, 22.6 and 22.5 us -- longer
+// slices keep each warp's two-stage cp.async pipeline full -- while the
+// 256-token step did not move.  Pack keeps 32 (it has no such pipeline).
+constexpr int kSliceWarpsPerSm = 16;
 
 __device__ __forceinline__ SrcEntry read_entry(const SrcEntry *e) {
   uint4 v;
@@ -433,7 +439,7 @@ cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
     a.coef = coef;
     a.src_cap = L.capacity;
     a.nvec = (int)(a.rb_in / 16);
-    row_slices(a.n_items, a.nvec, ctx.num_sms, a.slices, a.svec);
+    row_slices(a.n_items, a.nvec, ctx.num_sms, a.slices, a.svec, kSliceWarpsPerSm);
     return launch_fanin(a, dtype, out_dtype, ctx, s);
   }
   // both reverse hops in one pass per token
@@ -452,7 +458,7 @@ cudaError_t launch_combine(const void *y, int dtype, int H, const moe_layout &L,
   b.cap1 = L.capacity_hop1;
   b.nvec = (int)(b.rb_in / 16);
   if (b.T == 0) return cudaSuccess;
-  row_slices(b.T, b.nvec, ctx.num_sms, b.slices, b.svec);
+  row_slices(b.T, b.nvec, ctx.num_sms, b.slices, b.svec, kSliceWarpsPerSm);
   if (dtype == MOE_F16) return launch_two_hop1<__half>(b, out_dtype, ctx, s);
   if (dtype == MOE_BF16) return launch_two_hop1<__nv_bfloat16>(b, out_dtype, ctx, s);
   return launch_two_hop1<float>(b, out_dtype, ctx, s);

@@ -111,10 +111,10 @@ inline cudaError_t set_smem_limit_once(Kern kern, int bytes, std::atomic<unsigne
 // Column slices per row for the one-warp-per-row copy kernels: few rows (the
 // decode regime) would leave most SMs idle and each warp walking its whole row
 // one dependent round trip after another, so a row is split into slices of
-// whole warp-widths (32 16-byte vectors each) until there are about 32 warps
-// per SM; many rows keep one slice each.
-inline void row_slices(long rows, int nvec, int num_sms, int &slices, int &svec) {
-  const long want = (long)num_sms * 32;
+// whole warp-widths (32 16-byte vectors each) until there are about
+// `warps_per_sm` warps per SM; many rows keep one slice each.
+inline void row_slices(long rows, int nvec, int num_sms, int &slices, int &svec, int warps_per_sm = 32) {
+  const long want = (long)num_sms * warps_per_sm;
   long s = rows > 0 ? (want + rows - 1) / rows : 1;
   const long cap = nvec / 32 > 0 ? nvec / 32 : 1;
   if (s > cap) s = cap;

@@ -11,6 +11,7 @@ __global__ void __launch_bounds__(256) replica_assign_kernel(
     const int *__restrict__ slots, int n_entries, const int *__restrict__ slot_rank, int S, int R,
     int *__restrict__ expert_slot, int *__restrict__ expert_rank, int *__restrict__ rank_active,
     DeviceCtx ctx) {
+  wait_prior_grids();
   extern __shared__ int4 sm_raw[];  // 16-byte aligned
   int *sm = reinterpret_cast<int *>(sm_raw);
   const MetroPlan P = metro_plan(E, n_entries, R);
@@ -30,8 +31,9 @@ cudaError_t launch_replica_assign(const int *counts, int E, const int *off, cons
   cudaError_t err = set_smem_limit_once(
       replica_assign_kernel, (int)(sizeof(int) * (assign_smem_ints(kMaxE, kMaxSlots, kMaxR) + kMaxE)), done);
   if (err != cudaSuccess) return err;
-  replica_assign_kernel<<<1, 256, smem, s>>>(counts, E, off, slots, n_entries, slot_rank, S, R,
-                                             expert_slot, expert_rank, rank_active, ctx);
+  err = launch_after_prior(replica_assign_kernel, dim3(1), dim3(256), smem, s, counts, E, off, slots,
+                           n_entries, slot_rank, S, R, expert_slot, expert_rank, rank_active, ctx);
+  if (err != cudaSuccess) return err;
   return count_launch(cudaGetLastError());
 }
 

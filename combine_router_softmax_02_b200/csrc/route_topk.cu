@@ -9,6 +9,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          int E, int k, int n_groups, int gpt,
                                                          int renorm, int *__restrict__ idx_out,
                                                          float *__restrict__ w_out, DeviceCtx ctx) {
+  wait_prior_grids();
   __shared__ __align__(16) float s_cv[8][32];  // per-warp candidate logits
   __shared__ int s_ce[8][32];       // and their experts
   const int lane = threadIdx.x & 31;
@@ -37,12 +38,10 @@ cudaError_t launch_epl(const float *logits, int T, int E, int k, int n_groups, i
   long blocks = (T + wpb - 1) / wpb;
   const long cap = (long)ctx.num_sms * 16;
   if (blocks > cap) blocks = cap;
-  if (E == 32 * EPL)
-    route_topk_kernel<EPL, true><<<(unsigned)blocks, wpb * 32, 0, s>>>(logits, T, E, k, n_groups,
-                                                                      gpt, renorm, idx, w, ctx);
-  else
-    route_topk_kernel<EPL, false><<<(unsigned)blocks, wpb * 32, 0, s>>>(logits, T, E, k, n_groups,
-                                                                       gpt, renorm, idx, w, ctx);
+  auto kern = E == 32 * EPL ? route_topk_kernel<EPL, true> : route_topk_kernel<EPL, false>;
+  cudaError_t err = launch_after_prior(kern, dim3((unsigned)blocks), dim3(wpb * 32), 0, s, logits, T, E, k,
+                                       n_groups, gpt, renorm, idx, w, ctx);
+  if (err != cudaSuccess) return err;
   return count_launch(cudaGetLastError());
 }
 

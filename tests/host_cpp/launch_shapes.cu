@@ -34,14 +34,15 @@ int main() {
   const int nvecs[] = {1, 16, 31, 32, 33, 512, 896, 4096};
   for (long rows : rows_)
     for (int nvec : nvecs)
-      for (int sms : {1, 148}) {
+      for (int sms : {1, 148})
+      for (int wps : {16, 32}) {
         int slices = 0, svec = 0;
-        moe::row_slices(rows, nvec, sms, slices, svec);
+        moe::row_slices(rows, nvec, sms, slices, svec, wps);
         if (slices < 1 || svec < 1) return fail("empty slicing", rows, nvec, sms);
         if ((long)slices * svec < nvec || (long)(slices - 1) * svec >= nvec)
           return fail("slices do not cover the row exactly", rows, nvec, slices);
         if (slices > 1 && svec % 32 != 0) return fail("a slice is not whole warp-widths", rows, nvec, svec);
-        if (rows >= 32L * sms && slices != 1) return fail("many rows should keep one slice", rows, nvec, slices);
+        if (rows >= (long)wps * sms && slices != 1) return fail("many rows should keep one slice", rows, nvec, slices);
         if ((long)rows * slices >= (1L << 31)) return fail("work items overflow 31 bits", rows, nvec, slices);
       }
   std::printf("ok\n");

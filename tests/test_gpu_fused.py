@@ -156,6 +156,13 @@ def test_one_launch_front_edges(moe, T, E, k, R, mode, rpg, extra):
                       np.array(slot_rank, np.int32))
     sep, one = run_one_launch(moe, cfg, logits, rm)
     assert_same_front(moe, cfg, sep, one)
+    # and against the oracle (the separate calls share the greedy's device code)
+    idx, _ = oracle.route_topk(logits, k)
+    counts = oracle.demand_hist(idx, E)
+    slot, er, act = oracle.replica_assign(counts, rm.replica_offsets, rm.replica_slots, rm.slot_rank, R)
+    assert np.array_equal(one.expert_slot.cpu().numpy(), slot)
+    assert np.array_equal(one.expert_rank.cpu().numpy(), er)
+    assert np.array_equal(one.rank_active.cpu().numpy(), act)
 
 
 def test_one_launch_front_zero_tokens(moe):

@@ -154,6 +154,59 @@ def test_assign_random_maps_with_ties(moe):
             assert np.array_equal(g, r.astype(np.int32)), trial
 
 
+def _random_map(rng, E, R, max_rep):
+    """Replica map with 1..max_rep replicas per expert on distinct random
+    ranks; slot ids shuffled so that they are not in expert order."""
+    nrep = rng.integers(1, min(R, max_rep) + 1, size=E)
+    reps = [rng.choice(R, size=int(n), replace=False) for n in nrep]
+    slot_rank = np.concatenate(reps).astype(np.int32)
+    S = slot_rank.shape[0]
+    perm = rng.permutation(S)
+    sr_by_slot = np.empty(S, np.int32)
+    sr_by_slot[perm] = slot_rank
+    off = np.zeros(E + 1, np.int32)
+    off[1:] = np.cumsum(nrep)
+    return off, perm.astype(np.int32), sr_by_slot
+
+
+@pytest.mark.parametrize("R", [1, 5, 8, 9, 16, 17, 32, 33, 64])
+def test_assign_small_replica_sets(moe, R):
+    """No expert with more than 4 replicas and at most 255 with a choice: the
+    one-thread walk, whose per-rank counters are bytes of 64-bit words (one
+    word up to 8 ranks, then 2, 4 and 8 words); demand with zeros and ties."""
+    rng = np.random.default_rng(100 + R)
+    for trial in range(8):
+        E = int(rng.integers(1, 400))
+        off, slots, sr = _random_map(rng, E, R, 4)
+        counts = rng.integers(0, 3, size=E).astype(np.int32)
+        got = _assign_dev(moe, counts, off, slots, sr, R)
+        assert moe.get_status() == 0
+        ref = oracle.replica_assign(counts, off, slots, sr, R)
+        for g, r in zip(got, ref):
+            assert np.array_equal(g, r.astype(np.int32)), (R, trial)
+
+
+@pytest.mark.parametrize("n_choice", [255, 256])
+def test_assign_choice_count_boundary(moe, n_choice):
+    """255 active experts with a choice take the one-thread walk, 256 the warp
+    walk; both give the greedy's result."""
+    rng = np.random.default_rng(n_choice)
+    E, R = 400, 16
+    nrep = np.ones(E, np.int64)
+    nrep[:n_choice] = 2
+    reps = [rng.choice(R, size=int(n), replace=False) for n in nrep]
+    sr = np.concatenate(reps).astype(np.int32)
+    off = np.zeros(E + 1, np.int32)
+    off[1:] = np.cumsum(nrep)
+    slots = np.arange(sr.shape[0], dtype=np.int32)
+    counts = np.ones(E, np.int32)
+    got = _assign_dev(moe, counts, off, slots, sr, R)
+    assert moe.get_status() == 0
+    ref = oracle.replica_assign(counts, off, slots, sr, R)
+    for g, r in zip(got, ref):
+        assert np.array_equal(g, r.astype(np.int32))
+
+
 def test_assign_active_expert_without_replica(moe):
     counts = [1, 2, 0]
     s, r, a = _assign_dev(moe, counts, [0, 1, 1, 2], [0, 1], [0, 1], 2)
