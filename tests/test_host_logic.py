@@ -61,3 +61,39 @@ def test_step_trace_two_hop_groups():
     assert hop1["bytes"] == 8 * b and hop1["group_bytes"] == [5 * b, 3 * b]
     assert [d["group"] for d in tr["rank_detail"]] == [0, 0, 1, 1]
     assert "calls_us" not in tr
+
+
+@pytest.mark.parametrize("name", ["c4", "c5"])
+def test_parallel_oracle_matches_serial(name):
+    """The all-cores CPU baseline runs the same oracle functions over disjoint
+    chunks in spawned processes: its packed rows and combined tokens equal a
+    single-process pass over the same sample."""
+    import numpy as np
+    import bench
+    import oracle
+    import workloads as W
+    cfg = W.CONFIGS[name]
+    sub, logits, x32, rm = bench.oracle_sample(cfg, 192, 0)
+    par = bench.ParallelOracle(sub, logits, x32, 2)
+    try:
+        rows = par.step(rm)
+        P = np.array(bench._shm_array(*par.p)[:rows])
+        out = np.array(bench._shm_array(*par.out))
+        idx, w = oracle.route_topk(logits, sub.k, sub.n_groups, sub.groups_per_token)
+        counts = oracle.demand_hist(idx, sub.E)
+        _, er, _ = oracle.replica_assign(counts, rm.replica_offsets, rm.replica_slots, rm.slot_rank, sub.R)
+        L = oracle.build_layout(idx, w, er, -(-sub.T // sub.R), sub.R, sub.mode, max(sub.ranks_per_group, 1))
+        assert rows == int(L["num_rows"])
+        if sub.mode == W.TWO_HOP:
+            p2 = oracle.pack(oracle.pack(x32, L["hop1_row_token"]), L["hop2_src_row"])
+            ref, _ = oracle.combine_two_hop(p2, L, L["row_coef"], sub.dtype)
+        else:
+            p2 = oracle.pack(x32, L["row_token"])
+            ref = oracle.combine(p2, L["token_rows"], L["row_coef"])
+        assert np.array_equal(P, p2)
+        assert np.array_equal(out, ref)
+    finally:
+        for shm in bench._SHM.values():  # this process's own views of the blocks
+            shm.close()
+        bench._SHM.clear()
+        par.close()
