@@ -51,12 +51,14 @@ struct FanoutArgs {
 // persistent grid of 2 blocks per SM cost 11%.
 //
 // Residency: fewer concurrent warps write fewer rows at a time, and the DRAM
-// then serves the writes faster.  A large launch (more than 8 blocks per SM;
-// a decode-sized one keeps every warp for latency) therefore reserves just over
-// a third of the SM's shared memory per block (unused), which holds it at 2
-// resident blocks per SM: 5 -> 2 blocks per SM took the 65536-token pack from
-// 1326 to 1302 us and the two-hop pack from 555 to 548 us (3 and 4 blocks per
-// SM fell in between, 1 block was slower on the first).
+// then serves the writes faster.  A launch of whole rows (one slice each) and
+// more than 2 blocks per SM therefore reserves just over a third of the SM's
+// shared memory per block (unused), which holds it at 2 resident blocks per
+// SM: 5 -> 2 blocks per SM took the 65536-token pack from 1326 to 1302 us and
+// the two-hop pack from 555 to 548 us (3 and 4 blocks per SM fell in between,
+// 1 block was slower on the first); on the 8192-token training workload the
+// same hold gives 78.6 -> 75.7 us.  A decode-sized launch (rows split into
+// column slices) keeps every warp for latency: the hold cost it 22.8 -> 24.2 us.
 constexpr int kU = 2;
 constexpr int kResidentBlocks = 2;
 
@@ -113,7 +115,7 @@ cudaError_t launch_kn(const FanoutArgs &a, const DeviceCtx &ctx, cudaStream_t s)
   const int wpb = 8;
   const long blocks = ((long)a.n_items * a.slices + wpb - 1) / wpb;
   int smem = 0;
-  if (blocks > 8L * ctx.num_sms && ctx.smem_per_sm > 0) {  // large launches only (decode keeps all warps)
+  if (a.slices == 1 && blocks > 2L * ctx.num_sms && ctx.smem_per_sm > 0) {  // whole rows (decode keeps all warps)
     smem = ctx.smem_per_sm / (kResidentBlocks + 1) + 1024;  // room for 2 blocks, not for 3
     static std::atomic<unsigned long long> smem_set{0};
     cudaError_t err = set_smem_limit_once(fanout_kernel<KM, NL, kU>, 160 * 1024, smem_set);
