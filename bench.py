@@ -442,7 +442,7 @@ def kernel_rooflines(cfg, per_us, bytes_, peak):
     return out
 
 
-def steps_for(probe_ms: float, min_s: float, floor: int, cap: int = 40000) -> int:
+def steps_for(probe_ms: float, min_s: float, floor: int, cap: int = 100000) -> int:
     """Passes that fill at least `min_s` seconds at `probe_ms` per pass."""
     if probe_ms <= 0:
         return floor
