@@ -135,7 +135,8 @@ MOE_API int moe_demand_hist(const int32_t *topk_idx, int32_t T, int32_t k, int32
                     int32_t *counts, moe_stream_t stream);
 
 /*
- * METRO greedy replica assignment (one CTA).  Source: same page, sections
+ * METRO greedy replica assignment (one CTA; the serial part walks only the
+ * experts with more than one valid replica).  Source: same page, sections
  * "changes the routing information" and "Add the expert-weight traffic term":
  * each active expert goes to one of its replicas on the rank with the fewest
  * already-activated experts.  Experts are visited in ascending id; ties go to
@@ -163,7 +164,9 @@ MOE_API size_t moe_layout_workspace_size(int32_t T, int32_t k, int32_t E, int32_
 /*
  * Stable per-destination row layout (one cooperative launch: per-block bin
  * counts, a bounded grid barrier, then each block's prefix from the count
- * table and its rows).
+ * table and its rows; at most 512 tokens in the DEDUP and TWO_HOP modes take
+ * one pass instead, every block counting every token, with no barrier and
+ * without touching the workspace).
  * Sources: the AllToAll(-v) destination chunks of "METRO AllGather vs AllToAll
  * for MoE decode", sections "Work the 8-GPU payload example" and "Distinguish
  * METRO from backend names"; the single-send dispatcher of the ainewsletter
@@ -294,14 +297,16 @@ MOE_API int moe_route_layout_single_replica(
  * MoE decode", section "changes the routing information" (every rank computes
  * the global routing, the demand vector and the assignment: at decode sizes
  * their launch cost is what the global information costs).  One cooperative
- * kernel routes the tokens and counts the demand vector, one block runs the
- * METRO greedy over it, and every block then builds its part of the layout,
- * with grid barriers between the phases.  Every output equals that of the four
- * separate calls.  Arguments as in those calls; the workspace is
- * moe_layout_workspace_size() bytes as for moe_build_layout.  Returns
- * MOE_ERR_UNSUPPORTED, before anything is launched, if one block's shared
- * memory cannot hold the replica map and the layout bins (within the limits of
- * moe_replica_assign and moe_build_layout they take at most 139 KB).
+ * kernel routes the tokens and counts the demand vector; after a grid barrier
+ * every block runs the METRO greedy over it (the same deterministic result in
+ * each, written out by block 0) and builds its part of the layout, with one
+ * more grid barrier unless the layout takes one pass (at most 512 tokens,
+ * DEDUP or TWO_HOP).  Every output equals that of the four separate calls.
+ * Arguments as in those calls; the workspace is moe_layout_workspace_size()
+ * bytes as for moe_build_layout.  Returns MOE_ERR_UNSUPPORTED, before anything
+ * is launched, if one block's shared memory cannot hold the replica map and
+ * the layout bins (within the limits of moe_replica_assign and
+ * moe_build_layout they take at most 173 KB).
  */
 MOE_API int moe_route_assign_layout(
     const float *logits, int32_t T, int32_t E, int32_t k, int32_t n_groups, int32_t groups_per_token,
