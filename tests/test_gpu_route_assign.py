@@ -56,6 +56,59 @@ def test_route_edges(moe, T, E, k, G, gpt, renorm, ties):
     assert_weights(w_d.cpu().numpy(), w, logits, idx, renormalize=bool(renorm))
 
 
+@pytest.mark.parametrize("E,k,renorm,ties", [
+    (64, 6, 0, False),                  # the training workload's shape
+    (64, 8, 1, True),
+    (128, 1, 0, False),
+    (128, 8, 0, True),
+    (256, 8, 0, False),                 # the prefill workload's shape
+    (256, 8, 1, True),
+    (256, 3, 0, True),
+    (256, 7, 0, False),
+])
+def test_route_per_thread_kernel(moe, E, k, renorm, ties):
+    """Large token sets of these shapes (256 tokens per SM and more) take the
+    one-thread-per-token kernel; its picks and weights are bit-identical to the
+    one-warp-per-token kernel's, which runs on token sets below the threshold
+    (2000-token slices of the same logits) and on logits that are not 16-byte
+    aligned."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    T = 256 * sms + 77                  # a ragged last block of 32 tokens
+    rng = np.random.default_rng(E * 10 + k)
+    if ties:
+        logits = (rng.integers(-2, 3, size=(T, E)) * 0.5).astype(np.float32)
+        logits[::5] = 0.0
+        logits[1::7, ::3] = -0.0
+    else:
+        logits = rng.standard_normal((T, E)).astype(np.float32) * 3
+    dev = to_dev(logits)
+    idx_d, w_d = moe.route_topk(dev, k, 0, 0, bool(renorm))
+    assert moe.get_status() == 0
+    idx, w = oracle.route_topk(logits, k, 0, 0, bool(renorm))
+    idx_h, w_h = idx_d.cpu().numpy(), w_d.cpu().numpy()
+    assert np.array_equal(idx_h, idx)
+    assert_weights(w_h, w, logits, idx, renormalize=bool(renorm))
+    for t0 in range(0, T, 2000):
+        i_s, w_s = moe.route_topk(dev[t0:t0 + 2000], k, 0, 0, bool(renorm))
+        assert np.array_equal(i_s.cpu().numpy(), idx_h[t0:t0 + 2000])
+        assert np.array_equal(w_s.cpu().numpy().view(np.uint32), w_h[t0:t0 + 2000].view(np.uint32))
+    flat = torch.empty(T * E + 1, dtype=torch.float32, device="cuda")
+    shifted = flat[1:].view(T, E)
+    shifted.copy_(dev)
+    i_m, w_m = moe.route_topk(shifted, k, 0, 0, bool(renorm))
+    assert moe.get_status() == 0
+    assert np.array_equal(i_m.cpu().numpy(), idx_h)
+    assert np.array_equal(w_m.cpu().numpy().view(np.uint32), w_h.view(np.uint32))
+
+
+def test_route_per_thread_kernel_nonfinite(moe):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    lg = np.random.default_rng(5).standard_normal((256 * sms + 3, 256)).astype(np.float32)
+    lg[256 * sms + 1, 200] = np.inf     # in the ragged last block
+    moe.route_topk(to_dev(lg), 8)
+    assert moe.get_status() == 6            # MOE_ERR_BAD_INPUT
+
+
 def test_route_group_fixtures(moe):
     g = pins.golden("p4_group_limited.json")
     for c in g["cases"]:
