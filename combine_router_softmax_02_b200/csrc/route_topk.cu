@@ -4,10 +4,11 @@
 // collectives (the maximum, the butterfly sum, the k rounds for the candidate
 // bound, the compaction ballots) cost about 600 warp instructions a token, so
 // on a large token set it runs at the issue limit, far below the memory bound.
-// For the common shapes (E = 64, 128 or 256 experts, k <= 8, no group limit)
-// a second kernel gives each token a thread instead: a warp stages 32 tokens'
-// logit rows in shared memory and every lane routes its own token with plain
-// per-thread arithmetic, about a fifth of the instructions.  Its results are
+// For the common shapes (E = 64, 128 or 256 experts, k <= 8, no group limit
+// or groups of whole sixteenths of the experts) a second kernel gives each
+// token a thread instead: a warp streams 32 tokens' logit rows through shared
+// memory and every lane routes its own token with plain per-thread
+// arithmetic, well under half the instructions.  Its results are
 // bit-identical to the warp kernel's: the same maximum, the softmax sum added
 // in the same order (lane l's running sum over experts l, l + 32, ... and the
 // butterfly's pairing of the 32 partial sums, reproduced in registers), the
@@ -65,6 +66,20 @@ __device__ __forceinline__ float butterfly_sum(float (&a)[32]) {
   return a[0];
 }
 
+// One stage of a bitonic sort of 16 values into descending order: pairs
+// (i, i + D) inside blocks of SIZE, descending where i & SIZE is clear.
+template <int SIZE, int D>
+__device__ __forceinline__ void bitonic_stage(float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (!(i & D)) {
+      const float hi = fmaxf(x[i], x[i | D]), lo = fminf(x[i], x[i | D]);
+      const bool desc = !(i & SIZE) || SIZE == 16;
+      x[i] = desc ? hi : lo;
+      x[i | D] = desc ? lo : hi;
+    }
+}
+
 // Routes the T tokens, 32 to a block (one warp).  The block streams its
 // tokens' logits through shared memory in 32-expert columns (32 tokens x 32
 // experts, 4 KB), three columns in flight (cp.async), the row stride padded to
@@ -72,11 +87,16 @@ __device__ __forceinline__ float butterfly_sum(float (&a)[32]) {
 // column of eight rows fall in distinct banks; the small tiles leave room for
 // many resident warps.  The columns go by twice (the second time mostly from
 // L2), and lane l routes token t0 + l:
-//   1. first pass: the non-finite check, the maximum m and the maxima of 8
-//      chunks of E/8 experts; tau = the k-th largest chunk maximum bounds the
-//      k-th largest logit from below (k chunks hold an element >= tau);
+//   1. first pass: the non-finite check, the maximum m and the maxima of 16
+//      chunks of E/16 experts.  Under a group limit (groups of whole chunks)
+//      a group's score is the largest of its chunks' maxima, and the token keeps
+//      its best groups_per_token groups (gpt rounds of a scan in chunk order,
+//      ties to the lower group); tau = the k-th largest maximum of the kept
+//      chunks (a sorting network) bounds the k-th largest kept logit from below
+//      (k kept chunks hold an element >= tau; -inf when fewer than k are kept);
 //   2. second pass: expert e adds e^(v - m) to partial sum e % 32 (the warp
-//      kernel's lane e % 32) and, when v >= tau, is a candidate; each column's
+//      kernel's lane e % 32; the softmax is over every expert) and, when it is
+//      kept and v >= tau, is a candidate; each column's
 //      candidates go, in ascending expert order, through an insertion network
 //      that keeps the k best order keys: a candidate goes in before the first
 //      entry with a strictly smaller key and every entry after it shifts down
@@ -90,13 +110,14 @@ constexpr int kColTiles = 3;    // column tiles in flight
 
 template <int E, int KM>
 __global__ void __launch_bounds__(kRowTokens, 16) route_rows_kernel(const float *__restrict__ logits, int T,
-                                                                int k, int renorm,
+                                                                int k, int n_groups, int gpt, int renorm,
                                                                 int *__restrict__ idx_out,
                                                                 float *__restrict__ w_out, DeviceCtx ctx) {
   static_assert(E % 32 == 0 && E <= 256 && KM <= 8, "the per-thread router's shapes");
-  constexpr int NC = E / 32;   // columns
-  constexpr int CH = E / 8;    // experts per chunk of the bound
-  constexpr int CPC = 32 / CH; // chunks per column
+  constexpr int NC = E / 32;    // columns
+  constexpr int NCH = 16;       // chunks of the bound
+  constexpr int CH = E / NCH;   // experts per chunk
+  constexpr int CPC = 32 / CH;  // chunks per column
   __shared__ __align__(16) float s_col[kColTiles][kRowTokens * kColStride];
   wait_prior_grids();
   const int lane = threadIdx.x;
@@ -119,9 +140,10 @@ __global__ void __launch_bounds__(kRowTokens, 16) route_rows_kernel(const float 
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
 
-  float z = 0.0f, cm[8], m = 0.0f, tau = 0.0f;
+  float z = 0.0f, cm[NCH], m = 0.0f, tau = 0.0f;
+  uint32_t keep = (1u << NCH) - 1;  // chunks kept by the group limit
 #pragma unroll
-  for (int c = 0; c < 8; ++c) cm[c] = -INFINITY;
+  for (int c = 0; c < NCH; ++c) cm[c] = -INFINITY;
   float acc[32];
 #pragma unroll
   for (int l = 0; l < 32; ++l) acc[l] = 0.0f;
@@ -155,27 +177,71 @@ __global__ void __launch_bounds__(kRowTokens, 16) route_rows_kernel(const float 
         cmax[4 * q / CH] = fmaxf(cmax[4 * q / CH], fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) cm[i] = (i / CPC == step) ? cmax[i % CPC] : cm[i];
+      for (int i = 0; i < NCH; ++i) cm[i] = (i / CPC == step) ? cmax[i % CPC] : cm[i];
       if (step == NC - 1) {
         if (lane < nt && !(z == 0.0f)) set_status(ctx.status, MOE_ERR_BAD_INPUT);
         float mx = cm[0];
 #pragma unroll
-        for (int c = 1; c < 8; ++c) mx = fmaxf(mx, cm[c]);
+        for (int c = 1; c < NCH; ++c) mx = fmaxf(mx, cm[c]);
         // the warp kernel's maximum: the largest order key of the lane
         // maxima, a lane whose maximum is -inf counting as key 0
         m = route::key_value(mx == -INFINITY ? 0u : route::order_key(mx));
-        tau = cm[0];
+        if (gpt > 0 && gpt < n_groups) {  // n_groups divides 16: groups of whole chunks
+          const int cpg = NCH / n_groups;
+          float gm[NCH];  // each chunk's group score
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          int rank = 0;
+          for (int i = 0; i < NCH; ++i) gm[i] = cm[i];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) rank += (cm[j] > cm[i] || (cm[j] == cm[i] && j < i)) ? 1 : 0;
-          tau = rank == k - 1 ? cm[i] : tau;
+          for (int ld = 0; ld < 4; ++ld) {  // NCH = 2^4
+            const int d = 1 << ld;
+            if (d < cpg)
+#pragma unroll
+              for (int i = 0; i < NCH; ++i)
+                if (!(i & d)) {
+                  const float g2 = fmaxf(gm[i], gm[i | d]);
+                  gm[i] = g2;
+                  gm[i | d] = g2;
+                }
+          }
+          keep = 0;
+#pragma unroll 1
+          for (int r = 0; r < gpt; ++r) {  // the best group left; ties to the lower one
+            float best = -INFINITY;
+            int bi = -1;
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) {
+              const bool take = !(keep >> i & 1u) && (bi < 0 || gm[i] > best);
+              best = take ? gm[i] : best;
+              bi = take ? i : bi;
+            }
+            keep |= ((1u << cpg) - 1u) << (bi & ~(cpg - 1));
+          }
         }
+        // tau: the k-th largest kept chunk maximum (bitonic sort, descending)
+        float x[NCH];
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) x[i] = (keep >> i & 1u) ? cm[i] : -INFINITY;
+        bitonic_stage<2, 1>(x);
+        bitonic_stage<4, 2>(x);
+        bitonic_stage<4, 1>(x);
+        bitonic_stage<8, 4>(x);
+        bitonic_stage<8, 2>(x);
+        bitonic_stage<8, 1>(x);
+        bitonic_stage<16, 8>(x);
+        bitonic_stage<16, 4>(x);
+        bitonic_stage<16, 2>(x);
+        bitonic_stage<16, 1>(x);
+        tau = x[0];  // x[k - 1], as the minimum of the first k (no indexed read)
+#pragma unroll
+        for (int r = 1; r < KM; ++r) tau = r < k ? fminf(tau, x[r]) : tau;
       }
     } else {
       // 2: partial sums in lane order, candidates through the insertion network
       const int col = step - NC;
+      uint32_t colkeep = 0;  // this column's experts in kept chunks
+#pragma unroll
+      for (int c = 0; c < CPC; ++c)
+        colkeep |= ((keep >> (col * CPC + c)) & 1u) ? ((1u << CH) - 1u) << (c * CH) : 0u;
       uint32_t cand = 0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -187,6 +253,7 @@ __global__ void __launch_bounds__(kRowTokens, 16) route_rows_kernel(const float 
         cand |= (x.x >= tau ? 1u : 0u) << (4 * q) | (x.y >= tau ? 2u : 0u) << (4 * q) |
                 (x.z >= tau ? 4u : 0u) << (4 * q) | (x.w >= tau ? 8u : 0u) << (4 * q);
       }
+      cand &= colkeep;
       while (cand) {
         const int l = __ffs(cand) - 1;
         cand &= cand - 1;
@@ -233,19 +300,21 @@ __global__ void __launch_bounds__(kRowTokens, 16) route_rows_kernel(const float 
 }
 
 // The per-thread router when it applies: E = 64, 128 or 256, k <= 8, no group
-// limit, 16-byte aligned logits, and tokens for at least 8 warps on every SM
-// (37888 on 148 SMs).  With fewer, too few warps share an SM to hide each
-// other's latency: on the 8192-token training workload (E = 64) it took
-// 11.4 us against the warp kernel's 10.7; on the 65536-token prefill workload
-// (E = 256) 39.9 against 46.8.
-constexpr int kRowMinWarpsPerSm = 8;
+// limit or groups of whole chunks (n_groups dividing 16), 16-byte aligned
+// logits, and tokens for at least 4 warps on every SM (18944 on 148 SMs).
+// With fewer, too few warps share an SM to hide each other's latency: on the
+// 8192-token training workload (E = 64, under 2 warps per SM) an earlier
+// version took 11.4 us against the warp kernel's 10.7.  On the 32768-token
+// two-hop workload (E = 128, 8 groups, 7 warps per SM) it takes 23.0 us against
+// 31.8, on the 65536-token prefill workload (E = 256) 36.0 against 47.4.
+constexpr int kRowMinWarpsPerSm = 4;
 
 template <int E>
-cudaError_t launch_rows(const float *logits, int T, int k, int renorm, int *idx, float *w,
-                        const DeviceCtx &ctx, cudaStream_t s) {
+cudaError_t launch_rows(const float *logits, int T, int k, int n_groups, int gpt, int renorm, int *idx,
+                        float *w, const DeviceCtx &ctx, cudaStream_t s) {
   const long blocks = ((long)T + kRowTokens - 1) / kRowTokens;
   cudaError_t err = launch_after_prior(route_rows_kernel<E, 8>, dim3((unsigned)blocks), dim3(kRowTokens), 0,
-                                       s, logits, T, k, renorm, idx, w, ctx);
+                                       s, logits, T, k, n_groups, gpt, renorm, idx, w, ctx);
   if (err != cudaSuccess) return err;
   return count_launch(cudaGetLastError());
 }
@@ -271,11 +340,11 @@ cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int n_gr
                               cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const bool limit = gpt > 0 && gpt < n_groups;
-  if ((long)T >= (long)kRowMinWarpsPerSm * kRowTokens * ctx.num_sms && k <= 8 && !limit &&
-      ((uintptr_t)logits & 15u) == 0) {
-    if (E == 64) return launch_rows<64>(logits, T, k, renorm, idx, w, ctx, s);
-    if (E == 128) return launch_rows<128>(logits, T, k, renorm, idx, w, ctx, s);
-    if (E == 256) return launch_rows<256>(logits, T, k, renorm, idx, w, ctx, s);
+  if ((long)T >= (long)kRowMinWarpsPerSm * kRowTokens * ctx.num_sms && k <= 8 &&
+      (!limit || 16 % n_groups == 0) && ((uintptr_t)logits & 15u) == 0) {
+    if (E == 64) return launch_rows<64>(logits, T, k, n_groups, gpt, renorm, idx, w, ctx, s);
+    if (E == 128) return launch_rows<128>(logits, T, k, n_groups, gpt, renorm, idx, w, ctx, s);
+    if (E == 256) return launch_rows<256>(logits, T, k, n_groups, gpt, renorm, idx, w, ctx, s);
   }
   const int epl = (E + 31) / 32;
   if (epl <= 1) return launch_epl<1>(logits, T, E, k, n_groups, gpt, renorm, idx, w, ctx, s);

@@ -105,9 +105,9 @@ typedef struct moe_layout {
 
 /*
  * Router softmax + top-k.  One token per warp; large token sets (at least
- * 256 tokens per SM) with E = 64, 128 or 256, k <= 8, no group limit and
- * 16-byte aligned logits take one token per thread instead, with bit-identical
- * results.
+ * 128 tokens per SM) with E = 64, 128 or 256, k <= 8, no group limit or
+ * n_groups dividing 16, and 16-byte aligned logits take one token per thread
+ * instead, with bit-identical results.
  * Source: "METRO AllGather vs AllToAll for MoE decode" (fanout.sh), section
  * "changes the routing information": every rank computes the top-k expert
  * choices of the full gathered token set.  Group-limited routing: TerraceMoE

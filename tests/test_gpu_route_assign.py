@@ -56,25 +56,32 @@ def test_route_edges(moe, T, E, k, G, gpt, renorm, ties):
     assert_weights(w_d.cpu().numpy(), w, logits, idx, renormalize=bool(renorm))
 
 
-@pytest.mark.parametrize("E,k,renorm,ties", [
-    (64, 6, 0, False),                  # the training workload's shape
-    (64, 8, 1, True),
-    (128, 1, 0, False),
-    (128, 8, 0, True),
-    (256, 8, 0, False),                 # the prefill workload's shape
-    (256, 8, 1, True),
-    (256, 3, 0, True),
-    (256, 7, 0, False),
+@pytest.mark.parametrize("E,k,G,gpt,renorm,ties", [
+    (64, 6, 0, 0, 0, False),            # the training workload's shape
+    (64, 8, 0, 0, 1, True),
+    (128, 1, 0, 0, 0, False),
+    (128, 8, 0, 0, 0, True),
+    (256, 8, 0, 0, 0, False),           # the prefill workload's shape
+    (256, 8, 0, 0, 1, True),
+    (256, 3, 0, 0, 0, True),
+    (256, 7, 0, 0, 0, False),
+    (128, 8, 8, 4, 0, False),           # the two-hop workload's shape: 8 groups, keep 4
+    (128, 8, 8, 4, 0, True),
+    (256, 8, 4, 2, 1, True),            # groups of 4 chunks
+    (64, 6, 16, 5, 0, False),           # groups of one chunk
+    (256, 8, 16, 3, 0, True),
+    (128, 2, 2, 1, 0, True),
+    (256, 8, 32, 4, 0, False),          # 32 groups: not whole chunks, the warp kernel
 ])
-def test_route_per_thread_kernel(moe, E, k, renorm, ties):
-    """Large token sets of these shapes (256 tokens per SM and more) take the
+def test_route_per_thread_kernel(moe, E, k, G, gpt, renorm, ties):
+    """Large token sets of these shapes (128 tokens per SM and more) take the
     one-thread-per-token kernel; its picks and weights are bit-identical to the
     one-warp-per-token kernel's, which runs on token sets below the threshold
     (2000-token slices of the same logits) and on logits that are not 16-byte
     aligned."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     T = 256 * sms + 77                  # a ragged last block of 32 tokens
-    rng = np.random.default_rng(E * 10 + k)
+    rng = np.random.default_rng(E * 10 + k + G)
     if ties:
         logits = (rng.integers(-2, 3, size=(T, E)) * 0.5).astype(np.float32)
         logits[::5] = 0.0
@@ -82,20 +89,20 @@ def test_route_per_thread_kernel(moe, E, k, renorm, ties):
     else:
         logits = rng.standard_normal((T, E)).astype(np.float32) * 3
     dev = to_dev(logits)
-    idx_d, w_d = moe.route_topk(dev, k, 0, 0, bool(renorm))
+    idx_d, w_d = moe.route_topk(dev, k, G, gpt, bool(renorm))
     assert moe.get_status() == 0
-    idx, w = oracle.route_topk(logits, k, 0, 0, bool(renorm))
+    idx, w = oracle.route_topk(logits, k, G, gpt, bool(renorm))
     idx_h, w_h = idx_d.cpu().numpy(), w_d.cpu().numpy()
     assert np.array_equal(idx_h, idx)
     assert_weights(w_h, w, logits, idx, renormalize=bool(renorm))
     for t0 in range(0, T, 2000):
-        i_s, w_s = moe.route_topk(dev[t0:t0 + 2000], k, 0, 0, bool(renorm))
+        i_s, w_s = moe.route_topk(dev[t0:t0 + 2000], k, G, gpt, bool(renorm))
         assert np.array_equal(i_s.cpu().numpy(), idx_h[t0:t0 + 2000])
         assert np.array_equal(w_s.cpu().numpy().view(np.uint32), w_h[t0:t0 + 2000].view(np.uint32))
     flat = torch.empty(T * E + 1, dtype=torch.float32, device="cuda")
     shifted = flat[1:].view(T, E)
     shifted.copy_(dev)
-    i_m, w_m = moe.route_topk(shifted, k, 0, 0, bool(renorm))
+    i_m, w_m = moe.route_topk(shifted, k, G, gpt, bool(renorm))
     assert moe.get_status() == 0
     assert np.array_equal(i_m.cpu().numpy(), idx_h)
     assert np.array_equal(w_m.cpu().numpy().view(np.uint32), w_h.view(np.uint32))
