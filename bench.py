@@ -255,6 +255,7 @@ EXTRA_RUNS = (
     ("c5 two-hop", "c5", {}, False, False, True),
     ("c3 training, correlated placement", "c3", {}, False, False, False),
     ("c3 training, round-robin placement", "c3", {"placement": "roundrobin"}, False, False, False),
+    ("c3 training, correlated placement, one-launch front end", "c3", {}, True, False, False),
     ("c1 METRO toy decode", "c1", {}, False, False, False),
     ("c1 METRO toy decode, one-launch front end, CUDA graph", "c1", {}, True, True, False),
     ("c2 MoE decode", "c2", {}, False, False, False),
