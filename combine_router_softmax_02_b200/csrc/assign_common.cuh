@@ -328,23 +328,30 @@ __device__ __forceinline__ void metro_solve(const int *counts, int E, int R, int
   __syncthreads();
 
   // 2: forced experts of earlier chunks per (chunk, rank), row C = all
-  // chunks; and the ascending list of active choice experts, each chunk's
-  // experts after those of the earlier chunks.  Direct sums of at most 32
-  // independent loads: no serial chain.
-  for (int x = tid; x < (C + 1) * R; x += blockDim.x) {
-    const int c = x / R, r = x - c * R;
-    int run = 0;
-    for (int c2 = 0; c2 < c; ++c2) run += __popc(s_mask[c2 * R + r]);
-    s_pre[x] = run;
-  }
-  for (int c = tid; c <= C; c += blockDim.x) {
-    int base = 0;
-    for (int c2 = 0; c2 < c; ++c2) base += __popc((unsigned)s_cmask[c2]);
-    if (c == C) {
-      sm[P.nlist] = base;
-    } else {
-      for (unsigned m = (unsigned)s_cmask[c]; m; m &= m - 1) s_list[base++] = c * 32 + __ffs(m) - 1;
+  // chunks, and the ascending list of active choice experts, each chunk's
+  // experts after those of the earlier chunks: exclusive warp scans over the
+  // chunks (lane c holds chunk c; C <= 32), one per rank and one for the list.
+  auto warp_scan = [&](int v) {  // inclusive prefix sum over the lanes
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int t = __shfl_up_sync(kFull, v, d);
+      if (lane >= d) v += t;
     }
+    return v;
+  };
+  for (int r = warp; r < R; r += nwarps) {
+    const int v = lane < C ? __popc(s_mask[lane * R + r]) : 0;
+    const int incl = warp_scan(v);
+    if (lane < C) s_pre[lane * R + r] = incl - v;
+    if (lane == C - 1) s_pre[C * R + r] = incl;
+  }
+  if (warp == nwarps - 1) {
+    const unsigned cm = lane < C ? (unsigned)s_cmask[lane] : 0u;
+    const int v = __popc(cm);
+    const int incl = warp_scan(v);
+    int base = incl - v;
+    for (unsigned m = cm; m; m &= m - 1) s_list[base++] = lane * 32 + __ffs(m) - 1;
+    if (lane == 31) sm[P.nlist] = incl;
   }
   __syncthreads();
 
