@@ -1,6 +1,7 @@
 """Host-side logic of the package that needs no GPU."""
 import pytest
 
+import workloads as W
 from combine_router_softmax_02_b200.path import token_ranges
 
 
@@ -97,3 +98,26 @@ def test_parallel_oracle_matches_serial(name):
             shm.close()
         bench._SHM.clear()
         par.close()
+
+
+def test_bench_extra_runs_are_well_formed():
+    """Every workload the default bench run measures beside the headline names
+    a config, applies only Config fields, carries a unique label, and asks for
+    a CUDA graph only together with the one-launch front end."""
+    import bench
+    labels = [r[0] for r in bench.EXTRA_RUNS]
+    assert len(labels) == len(set(labels))
+    for label, name, over, fused, graph, e2e in bench.EXTRA_RUNS:
+        assert name in W.CONFIGS, label
+        cfg = W.CONFIGS[name].with_(**over)     # raises on an unknown field
+        assert cfg.name == name
+        assert not graph or fused, label
+        assert isinstance(e2e, bool)
+
+
+def test_bench_steps_for_bounds():
+    import bench
+    assert bench.steps_for(0.0, 1.0, 20) == 20
+    assert bench.steps_for(2.6, 1.0, 20) == 385      # ceil(1000 / 2.6)
+    assert bench.steps_for(0.001, 1.0, 20, cap=100000) == 100000
+    assert bench.steps_for(5000.0, 1.0, 20) == 20
